@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Throughput of the lookahead importance-scoring path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--cmax C]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on the host cores
+
+One step = speckv_score (row-LSE pass + column-sum pass) + topk_select (pool 7,
+top-C_max + window) + kv_compact over every unit of the workload, through the
+C ABI of libspeckv.so.  Default workload: the Qwen2.5-32B-shaped SpecKV pass at
+64K context (64 layers, 40/8 heads, head_dim 128, window 64, lookahead 128,
+C_max 256), seeded synthetic bf16 inputs resident in HBM (K and V are 8.6 GB
+each, far larger than the 126 MB L2, so no L2 flush is needed between steps).
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
+seed (units are independent, no data-path collective): weak scaling.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "KV-head-tokens scored+selected+compacted/s at 64K ctx"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--config", default=W.QWEN32B_64K.name,
+                    choices=[c.name for c in W.CONFIGS.values() if isinstance(c, W.SpecKVConfig)])
+    ap.add_argument("--cmax", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def config_of(args) -> W.SpecKVConfig:
+    import dataclasses
+    cfg = W.CONFIGS[args.config]
+    if args.cmax is not None:
+        cfg = dataclasses.replace(cfg, c_max=args.cmax)
+    return cfg
+
+
+def algorithmic_flops(cfg: W.SpecKVConfig) -> float:
+    """One Q.K^T product over the causally visible keys of every row:
+    2 * d * g * sum_i c_i per unit (each of the two passes does this once)."""
+    vis = sum(cfg.n_pre + i + 1 for i in range(cfg.n_window)) + cfg.n_lookahead * cfg.n_in
+    return 2.0 * cfg.head_dim * cfg.g * vis * cfg.units
+
+
+def algorithmic_bytes(cfg: W.SpecKVConfig) -> float:
+    """K read once, Q read once, scores written and read once, K and V rows of
+    the reduced cache read and written once."""
+    d = cfg.head_dim
+    per_unit = cfg.n_in * d * 2 + cfg.g * cfg.rows * d * 2 + 8 * cfg.n_pre + 4 * cfg.keep * d * 2
+    return per_unit * cfg.units
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained"), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- oracle timing
+def _oracle_unit_job(payload):
+    """Scores -> pool -> top-C_max + window -> gather, for one unit (fp64 oracle)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    qb, kb, vb, n_window, n_lookahead, c_max, pool = payload
+    s, p, idx = oracle.speckv_select_unit(qb, kb, n_window, n_lookahead, c_max, pool)
+    oracle.gather_rows(kb, idx)
+    oracle.gather_rows(vb, idx)
+    return int(idx.size)
+
+
+def time_oracle(units_payload, cores):
+    """Run the oracle on the given units over `cores` spawned processes; returns seconds."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(processes=cores) as pool:
+        pool.map(_oracle_unit_job, units_payload[:1])          # warm: import + build
+        t0 = time.perf_counter()
+        pool.map(_oracle_unit_job, units_payload, chunksize=1)
+        return time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_sample_payload(cfg, seed, n_units):
+    payload = []
+    for u in range(n_units):
+        qb, kb, vb = W.speckv_unit_numpy(cfg, seed, u)
+        payload.append((qb, kb, vb, cfg.n_window, cfg.n_lookahead, cfg.c_max, cfg.pool))
+    return payload
+
+
+def run_reference(args, cfg):
+    """--impl reference: the fp64 oracle on the host cores, same metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    cores = host_cores()
+    per_step = cores                     # one unit per core per step
+    payload = cpu_sample_payload(cfg, args.seed, per_step)
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    times = []
+    with ctx.Pool(processes=cores) as pool:
+        pool.map(_oracle_unit_job, payload[:1])
+        for s in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            pool.map(_oracle_unit_job, payload, chunksize=1)
+            if s >= args.warmup:
+                times.append(time.perf_counter() - t0)
+    step = sum(times) / len(times)
+    value = per_step * cfg.n_in / step
+    sample = (f"{per_step} units of {cfg.name} per step (one per core, seeded host inputs); "
+              f"full step = {cfg.units} units")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "KV-head-tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "units_per_step": per_step, "n_in": cfg.n_in,
+                   "c_max": cfg.c_max, "pool": cfg.pool},
+        "cpu_baseline": {"value": value, "unit": "KV-head-tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "KV-head-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- GPU arm
+def main():
+    args = parse()
+    cfg = config_of(args)
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from prompt_compression_b200 import build
+    build.build_library()
+    import prompt_compression_b200 as P
+    from prompt_compression_b200.pipeline import SpeckvBuffers
+
+    seed = args.seed + 1000 * rank
+    inp = W.speckv_inputs(cfg, seed=seed, device=dev)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    buf = SpeckvBuffers(q, k, v, cfg.n_window, cfg.c_max)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        P.speckv_compress(q, k, v, cfg.n_window, cfg.c_max, cfg.pool, buffers=buf, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, site = P.spk_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} at site {site} during warm-up")
+
+    # ---- timed region: K steps, events on the launching stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms_total / args.steps
+    value = world * cfg.kv_head_tokens * args.steps / (ms_total * 1e-3)
+
+    # ---- per-kernel timing: pass 1 alone (row LSE), then the whole score call
+    lse2 = torch.empty((cfg.units, cfg.g * cfg.rows), dtype=torch.float32, device=dev)
+
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    n_k = max(3, min(args.steps, 10))
+    ms_lse = timed(lambda: P.speckv_row_lse(q, k, cfg.n_window, lse2, stream=stream), n_k)
+    ms_score = timed(lambda: P.speckv_score(q, k, cfg.n_window, buf.scores, None, buf.ws_score,
+                                            stream=stream), n_k)
+    ms_topk = timed(lambda: P.topk_select(buf.scores, cfg.c_max, cfg.n_window, buf.idx, cfg.pool, None,
+                                          buf.ws_topk, stream=stream), n_k)
+    ms_compact = timed(lambda: P.kv_compact(k, v, buf.idx, buf.k_out, buf.v_out, 1, stream=stream), n_k)
+    ms_colsum = ms_score - ms_lse
+    st, site = P.spk_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} at site {site}")
+
+    peaks = load_peaks()
+    flops_pass = algorithmic_flops(cfg)
+    kernels = {
+        "score_lse_pass": {"ms": ms_lse, "tflops": flops_pass / (ms_lse * 1e-3) / 1e12},
+        "score_colsum_pass": {"ms": ms_colsum, "tflops": flops_pass / (ms_colsum * 1e-3) / 1e12},
+        "topk_select": {"ms": ms_topk},
+        "kv_compact": {"ms": ms_compact,
+                       "gbs": cfg.units * 4 * cfg.keep * cfg.head_dim * 2 / (ms_compact * 1e-3) / 1e9},
+    }
+    dom = "score_lse_pass" if ms_lse >= ms_colsum else "score_colsum_pass"
+    achieved = kernels[dom]["tflops"]
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            traffic = json.load(open(prof)).get(dom, {}).get(cfg.name)
+        except Exception:
+            traffic = None
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 burst",
+                "step_roofline_ms": max(2 * flops_pass / (peaks["bf16_tflops"] * 1e12),
+                                        algorithmic_bytes(cfg) / (peaks["hbm_gbs"] * 1e9)) * 1e3}
+    roofline["step_frac"] = roofline["step_roofline_ms"] / ms_step
+
+    # ---- e2e through the C ABI with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_over_ranks, barrier)
+
+    # ---- CPU baseline (oracle), rank 0 at N = 1 only
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cores = host_cores()
+        n_units = max(1, min(cores, 8))
+        payload = cpu_sample_payload(cfg, args.seed, n_units)
+        secs = time_oracle(payload, n_units)
+        cpu = {"value": n_units * cfg.n_in / secs, "unit": "KV-head-tokens/s", "cores": n_units,
+               "kind": "oracle",
+               "sample": f"{n_units} units of {cfg.name} (one per process, seeded host inputs), "
+                         f"{secs:.1f} s wall; the full step has {cfg.units} units"}
+
+    launches = 4 * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "KV-head-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "units": cfg.units, "layers": cfg.layers, "hq": cfg.hq,
+                   "hkv": cfg.hkv, "head_dim": cfg.head_dim, "n_in": cfg.n_in, "n_window": cfg.n_window,
+                   "n_lookahead": cfg.n_lookahead, "c_max": cfg.c_max, "pool": cfg.pool,
+                   "l2": "inputs larger than L2 (K, V 8.6 GB each at 64K); no flush",
+                   "parallelism": f"units sharded, {world} rank(s), no collective"},
+        "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
+        "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_over_ranks, barrier):
+    """Same metric end to end: each step copies Q, K, V from pinned host memory,
+    runs the three C-ABI calls, and copies the indices and compacted K/V back."""
+    import torch
+    from prompt_compression_b200.pipeline import SpeckvBuffers
+    need = (q.numel() + k.numel() + v.numel()) * 2
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    if avail is not None and avail < 2 * need:
+        return {"value": None, "unit": "KV-head-tokens/s", "skipped":
+                f"host RAM available {avail / 2**30:.0f} GiB < 2 x {need / 2**30:.0f} GiB of pinned inputs"}
+    hq_ = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+    hq_.copy_(q)
+    hk.copy_(k)
+    hv.copy_(v)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    buf = SpeckvBuffers(dq, dk, dv, cfg.n_window, cfg.c_max)
+    oi = torch.empty(buf.idx.shape, dtype=buf.idx.dtype, pin_memory=True)
+    ok_ = torch.empty(buf.k_out.shape, dtype=buf.k_out.dtype, pin_memory=True)
+    ov = torch.empty(buf.v_out.shape, dtype=buf.v_out.dtype, pin_memory=True)
+
+    def step():
+        dq.copy_(hq_, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        P.speckv_compress(dq, dk, dv, cfg.n_window, cfg.c_max, cfg.pool, buffers=buf, stream=stream)
+        oi.copy_(buf.idx, non_blocking=True)
+        ok_.copy_(buf.k_out, non_blocking=True)
+        ov.copy_(buf.v_out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b)) / args.e2e_steps
+    h2d = (q.numel() + k.numel() + v.numel()) * 2
+    d2h = oi.numel() * 4 + (ok_.numel() + ov.numel()) * 2
+    return {"value": world * cfg.kv_head_tokens / (ms * 1e-3), "unit": "KV-head-tokens/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": args.e2e_steps}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * speckv.h -- C ABI of the B200 (sm_100a) lookahead importance-scoring library.
+ *
+ * The method is "Draft-based Approximate Inference for LLMs" (paper notes,
+ * ICLR 2026, arXiv 2506.08373):
+ *   - section 关键设计, SpecKV: for every attention head, the queries of the
+ *     last n_window input tokens and of the n_lookahead draft (lookahead)
+ *     tokens attend to the input keys; the attention that the remaining input
+ *     keys receive estimates the importance of each KV pair; the top-C_max KV
+ *     pairs plus the window are kept.
+ *   - section 关键设计, SpecPC: draft attention A[layer][head][query][key] over
+ *     a large query window with weights that fall with distance from the end,
+ *     the first l_skip layers skipped, averaged first, then maximised.
+ *   - section 关键设计, SpecKV-PC: SpecPC first, then SpecKV on what it kept.
+ *   - section 损失函数 / 训练策略: SpecPC smooths scores with local pooling.
+ *
+ * Conventions for every entry point
+ *   - Tensor arguments are DEVICE pointers owned by the caller, contiguous in
+ *     the layouts given below, 16-byte aligned.  The library allocates no
+ *     memory: scratch space is the caller's `workspace`, whose size comes from
+ *     the matching *_workspace_size() query.
+ *   - bf16 means IEEE bfloat16 bit patterns (uint16_t); fp32 is float.
+ *   - All work is enqueued on `stream` (a cudaStream_t, passed as void*;
+ *     NULL = legacy default stream) and returns without host synchronisation.
+ *   - The return value is a spk_status.  Argument errors are detected on the
+ *     host and returned BEFORE anything is launched; spk_last_error() then
+ *     describes the problem (thread-local string).
+ *   - Errors found on the device (a bounded wait that timed out, an index
+ *     outside its range in kv_compact) are recorded in a device error word
+ *     that spk_device_error() reads; kernels never trap.
+ *   - Results are deterministic: the same inputs give bitwise identical
+ *     outputs (no floating-point atomics).
+ *   - Calls on the same stream are ordered; calls that share a workspace must
+ *     not run concurrently on different streams.
+ */
+#ifndef SPECKV_H
+#define SPECKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPK_OK = 0,
+  SPK_ERR_ARG = 1,          /* a null/misaligned pointer or an inconsistent shape */
+  SPK_ERR_UNSUPPORTED = 2,  /* a valid shape outside what the kernels implement */
+  SPK_ERR_WORKSPACE = 3,    /* workspace missing or smaller than *_workspace_size() */
+  SPK_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (see spk_last_error) */
+  SPK_ERR_TIMEOUT = 5       /* reported by spk_device_error: a device wait ran out */
+} spk_status;
+
+/* ------------------------------------------------------------------------
+ * SpecKV scoring (section 关键设计, SpecKV)
+ *
+ * A unit is one (batch element, layer, KV head); units are numbered
+ * u = (b * layers + l) * hkv + h.  Query head qh belongs to KV head qh / g,
+ * g = hq / hkv (GQA).  R = n_window + n_lookahead query rows per query head:
+ * row i < n_window is the window query at input position n_in - n_window + i
+ * and sees input keys 0 .. n_in - n_window + i (causal); row i >= n_window is
+ * a lookahead (draft) query and sees all n_in input keys.  Keys of the
+ * lookahead tokens are not input keys and are not part of the softmax.
+ *
+ *   q      bf16 [batch][layers][hq][R][head_dim]   (rows pre-scaled or not: see scale)
+ *   k      bf16 [batch][layers][hkv][n_in][head_dim]
+ *   scores fp32 [units][n_pre], n_pre = n_in - n_window:
+ *          scores[u][j] = sum over the g query heads of unit u and their R rows
+ *                         of softmax_j(scale * q_row . k_j)   (prefix keys only)
+ *   window_mass fp32 [units][n_window] or NULL: the same sum on the window keys
+ *          j = n_pre .. n_in-1 (every prefix and window column together sum to
+ *          g * R per unit, which makes it a conservation check).
+ *
+ * Supported: head_dim in {64, 128}; hq % hkv == 0; g * R <= 2048;
+ * 0 <= n_window <= n_in; R >= 1; scale > 0 and finite.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int batch, layers, hq, hkv, head_dim;
+  int n_in, n_window, n_lookahead;
+  float scale; /* multiplies q.k before the softmax (1.0 if q is pre-scaled) */
+} spk_speckv_shape;
+
+size_t speckv_workspace_size(const spk_speckv_shape* shape);
+
+spk_status speckv_score(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16,
+                        float* scores, float* window_mass, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Pass 1 alone (diagnostic): the log2-domain log-sum-exp of every query row,
+ * lse2[u][qh_local * R + i] = log2 sum_{visible j} 2^(scale*log2(e) * q.k_j),
+ * fp32 [units][g * R].  Same shapes and rules as speckv_score. */
+spk_status speckv_row_lse(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16,
+                          float* lse2, void* stream);
+
+/* ------------------------------------------------------------------------
+ * SpecPC scoring (section 关键设计, SpecPC)
+ *
+ * Per batch element b, the draft's last W = n_rows query positions: row i sits
+ * at position n_in + n_lookahead - 1 - W + i and sees input keys 0 .. that
+ * position (capped at n_in - 1).  For every query head qh and layer
+ * l >= l_skip, P[l][qh][i][j] is the causal softmax of scale * q . k_j.
+ *   S[qh][j] = ( sum_{l >= l_skip} sum_i w_i P[l][qh][i][j] ) / ( sum_i w_i * (layers - l_skip) )
+ *   scores[b][j] = max_qh S[qh][j]        for j in 0 .. n_in-1
+ *
+ *   q            bf16 [batch][layers][hq][W][head_dim]   (layers < l_skip are not read)
+ *   k            bf16 [batch][layers][hkv][n_in][head_dim]
+ *   row_weights  fp32 [W], device, oldest row first, w_i >= 0, sum > 0
+ *   scores       fp32 [batch][n_in]
+ *
+ * Supported: head_dim == 64; hq % hkv == 0; hq / hkv <= 16; (hq/hkv) * W <= 2048;
+ * 0 <= l_skip < layers; 1 <= W <= n_in + n_lookahead - 1; n_lookahead >= 1.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int batch, layers, l_skip, hq, hkv, head_dim;
+  int n_in, n_rows, n_lookahead;
+  float scale;
+} spk_specpc_shape;
+
+size_t specpc_workspace_size(const spk_specpc_shape* shape);
+
+spk_status specpc_score(const spk_specpc_shape* shape, const void* q_bf16, const void* k_bf16,
+                        const float* row_weights, float* scores, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* ------------------------------------------------------------------------
+ * Pooling + top-k selection (section 关键设计: keep the top-C_max KV pairs plus
+ * the window; section 损失函数 / 训练策略: local pooling keeps token runs)
+ *
+ * For each of `units` rows of n_cand candidate scores:
+ *   pooled[j] = max scores[t] over t in [j - r, j + r] ∩ [0, n_cand), r = pool_kernel / 2
+ *   selected  = the min(k, n_cand) largest pooled values; equal values are
+ *               taken lowest index first
+ *   idx[u]    = selected indices in ascending order, then the tail
+ *               n_cand, n_cand + 1, .., n_cand + n_tail - 1 (the kept window)
+ *
+ *   scores  fp32 [units][n_cand], finite (NaN order is unspecified; -0 == +0)
+ *   idx     int32 [units][min(k, n_cand) + n_tail]
+ *   pooled  fp32 [units][n_cand] or NULL
+ *
+ * Supported: pool_kernel odd >= 1; k >= 0; n_tail >= 0; n_cand >= 0.
+ * ------------------------------------------------------------------------ */
+size_t topk_workspace_size(int units, int n_cand);
+
+spk_status topk_select(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail,
+                       int32_t* idx, float* pooled, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * KV compaction (section 关键设计, SpecKV: the dropped cache keeps only the
+ * selected KV pairs)
+ *
+ *   k_out[u][t] = k[u][ idx[u / units_per_idx][t] ],  same for v
+ *   k, v         [units][n_src][head_dim] elements of elem_bytes bytes
+ *   idx          int32 [units / units_per_idx][n_idx], each in [0, n_src)
+ *   k_out, v_out [units][n_idx][head_dim]
+ * units_per_idx = 1 gives every unit its own index row; units_per_idx =
+ * layers * hkv shares one row across all (layer, KV head) of a batch element
+ * (SpecPC / SpecKV-PC).  v and v_out may both be NULL.  Rows are copied
+ * byte for byte.  An index outside [0, n_src) leaves that output row
+ * unwritten and records SPK_ERR_ARG in the device error word.
+ *
+ * Supported: head_dim * elem_bytes a multiple of 16; units % units_per_idx == 0.
+ * ------------------------------------------------------------------------ */
+spk_status kv_compact(const void* k, const void* v, int units, int n_src, int head_dim, int elem_bytes,
+                      const int32_t* idx, int n_idx, int units_per_idx, void* k_out, void* v_out,
+                      void* stream);
+
+/* ------------------------------------------------------------------------
+ * Errors
+ * ------------------------------------------------------------------------ */
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* spk_last_error(void);
+
+/* Synchronises the current device, then reports the first error recorded by a
+ * kernel since the last clear: *status = SPK_OK, SPK_ERR_TIMEOUT (a bounded
+ * device wait ran out; *site says where) or SPK_ERR_ARG (kv_compact index out
+ * of range).  clear != 0 resets the word.  Returns SPK_ERR_CUDA if the
+ * device could not be read. */
+spk_status spk_device_error(int* status, int* site, int clear);
+
+/* Self-test of the bounded waits: launches one kernel that waits on a barrier
+ * nothing will complete, with a limit of limit_ns nanoseconds (clamped to
+ * [1e3, 1e9]).  The kernel gives up, records SPK_ERR_TIMEOUT at site 999 and
+ * returns; read it with spk_device_error().  No GPU state is left behind. */
+spk_status spk_selftest_wait_timeout(long long limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPECKV_H */

@@ -1,0 +1,33 @@
+"""B200 (sm_100a) lookahead importance scoring: SpecKV / SpecPC scoring, pooling,
+top-k selection and KV compaction.
+
+This package is a thin binding over ``libspeckv.so`` (the C ABI declared in
+``include/speckv.h``).  The functions below marshal torch tensors into raw
+device pointers, sizes and a stream and call the C entry point of the same
+name; every step of the computation runs in the library's CUDA kernels.
+There is no CPU fallback: if the library is missing or cannot be loaded,
+every call raises.
+
+Method: "Draft-based Approximate Inference for LLMs" (paper notes, ICLR 2026),
+section 关键设计 (SpecKV, SpecPC, SpecKV-PC) and section 损失函数 / 训练策略
+(local pooling).
+"""
+from __future__ import annotations
+
+from .binding import (  # noqa: F401
+    SpeckvError, load_library, library_path,
+    speckv_workspace_size, speckv_score, speckv_row_lse,
+    specpc_workspace_size, specpc_score,
+    topk_workspace_size, topk_select, kv_compact,
+    spk_device_error, spk_selftest_wait_timeout,
+)
+from .pipeline import speckv_compress, specpc_select, cascade_compress  # noqa: F401
+
+__all__ = [
+    "SpeckvError", "load_library", "library_path",
+    "speckv_workspace_size", "speckv_score", "speckv_row_lse",
+    "specpc_workspace_size", "specpc_score",
+    "topk_workspace_size", "topk_select", "kv_compact",
+    "spk_device_error", "spk_selftest_wait_timeout",
+    "speckv_compress", "specpc_select", "cascade_compress",
+]

@@ -1,0 +1,57 @@
+"""Build libspeckv.so (the sm_100a kernels behind include/speckv.h) in-tree.
+
+    python -m prompt_compression_b200.build [--force]
+
+nvcc cross-compiles for sm_100a; no GPU is needed to build.
+"""
+from __future__ import annotations
+
+import glob
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+LIB = os.path.join(PKG, "libspeckv.so")
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17", "-rdc=true",
+    "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
+]
+
+
+def sources():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
+def _inputs():
+    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [
+        os.path.join(ROOT, "include", "speckv.h"), os.path.abspath(__file__)]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", "nvcc"):
+        if cand and (os.path.sep not in cand or os.path.exists(cand)):
+            return cand
+    return "nvcc"
+
+
+def build_library(force: bool = False, verbose: bool = False) -> str:
+    """Compile every .cu under csrc/ into prompt_compression_b200/libspeckv.so."""
+    if not force and os.path.exists(LIB):
+        newest = max(os.path.getmtime(p) for p in _inputs())
+        if os.path.getmtime(LIB) >= newest:
+            return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc()] + NVCC_FLAGS + ["-o", tmp] + sources()
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd, cwd=PKG)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build_library(force="--force" in sys.argv, verbose=True))

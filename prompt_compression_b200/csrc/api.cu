@@ -1,0 +1,366 @@
+// api.cu -- the extern "C" boundary declared in include/speckv.h.
+//
+// Host side only: validates arguments (before any launch), builds the TMA
+// tensor maps, picks the persistent grid and enqueues the kernels on the
+// caller's stream.  No allocation, no host synchronisation on the compute
+// paths.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/speckv.h"
+#include "common.cuh"
+#include "score.cuh"
+
+namespace spk {
+namespace {
+
+thread_local char g_msg[512] = "";
+
+spk_status fail(spk_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+spk_status ok() {
+  g_msg[0] = 0;
+  return SPK_OK;
+}
+
+spk_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SPK_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int num_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 148;
+  return sms;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 view [n_units][n_rows][head_dim] read in 128-row x 64-column
+// boxes with the 128-byte swizzle the UMMA descriptors expect; rows past
+// n_rows read as zero.
+spk_status make_map(CUtensorMap* map, const void* base, int head_dim, long long n_rows, long long n_units) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(SPK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(n_rows),
+                              static_cast<cuuint64_t>(n_units)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                 static_cast<cuuint64_t>(n_rows) * head_dim * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SPK_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return SPK_OK;
+}
+
+struct SpeckvGeom {
+  long long units, rows, n_pre;
+  int g, R;
+};
+
+spk_status check_speckv(const spk_speckv_shape* s, SpeckvGeom& g) {
+  if (s == nullptr) return fail(SPK_ERR_ARG, "shape is NULL");
+  if (s->batch < 1 || s->layers < 1 || s->hq < 1 || s->hkv < 1 || s->n_in < 1)
+    return fail(SPK_ERR_ARG, "batch, layers, hq, hkv and n_in must be >= 1");
+  if (s->hq % s->hkv != 0) return fail(SPK_ERR_ARG, "hq (%d) must be a multiple of hkv (%d)", s->hq, s->hkv);
+  if (s->n_window < 0 || s->n_lookahead < 0 || s->n_window > s->n_in)
+    return fail(SPK_ERR_ARG, "need 0 <= n_window <= n_in and n_lookahead >= 0");
+  if (s->n_window + s->n_lookahead < 1) return fail(SPK_ERR_ARG, "n_window + n_lookahead must be >= 1");
+  if (!(s->scale > 0.f) || !std::isfinite(s->scale)) return fail(SPK_ERR_ARG, "scale must be finite and > 0");
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(SPK_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", s->head_dim);
+  g.g = s->hq / s->hkv;
+  g.R = s->n_window + s->n_lookahead;
+  g.rows = static_cast<long long>(g.g) * g.R;
+  if (g.rows > kRowsMax)
+    return fail(SPK_ERR_UNSUPPORTED, "(hq/hkv) * (n_window + n_lookahead) = %lld exceeds %d", g.rows, kRowsMax);
+  g.units = static_cast<long long>(s->batch) * s->layers * s->hkv;
+  if (g.units * ((s->n_in + 255) / 256) > 0x7fffffffLL || g.units * 8 > 0x7fffffffLL)
+    return fail(SPK_ERR_UNSUPPORTED, "too many units");
+  g.n_pre = s->n_in - s->n_window;
+  return SPK_OK;
+}
+
+ScoreParams base_params(int head_dim, int n_in, const SpeckvGeom& g, int c0, float scale, int hkv,
+                        int layers_used, int layers_total, int l_skip) {
+  ScoreParams p;
+  memset(&p, 0, sizeof p);
+  p.head_dim = head_dim;
+  p.n_in = n_in;
+  p.rows = static_cast<int>(g.rows);
+  p.R = g.R;
+  p.c0 = c0;
+  p.c2 = scale * 1.4426950408889634f;
+  p.hkv = hkv;
+  p.layers_used = layers_used;
+  p.layers_total = layers_total;
+  p.l_skip = l_skip;
+  p.n_units = static_cast<int>(g.units);
+  return p;
+}
+
+spk_status run_lse(ScoreParams p, const CUtensorMap& qmap, const CUtensorMap& kmap, int head_dim,
+                   cudaStream_t stream) {
+  p.n_blocks = (p.rows + 255) / 256;
+  p.n_items = p.n_units * p.n_blocks;
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  cudaError_t e = launch_score(MODE_LSE, head_dim, qmap, kmap, p, grid, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "row-LSE launch");
+  return SPK_OK;
+}
+
+}  // namespace
+}  // namespace spk
+
+using namespace spk;
+
+extern "C" {
+
+const char* spk_last_error(void) { return g_msg; }
+
+size_t speckv_workspace_size(const spk_speckv_shape* s) {
+  SpeckvGeom g;
+  if (check_speckv(s, g) != SPK_OK) return 0;
+  return round_up(static_cast<size_t>(g.units) * g.rows * sizeof(float), 256);
+}
+
+static spk_status speckv_maps(const spk_speckv_shape* s, const void* q, const void* k, const SpeckvGeom& g,
+                              CUtensorMap* qmap, CUtensorMap* kmap) {
+  if (q == nullptr || k == nullptr) return fail(SPK_ERR_ARG, "q and k must be non-NULL device pointers");
+  if (!aligned16(q) || !aligned16(k)) return fail(SPK_ERR_ARG, "q and k must be 16-byte aligned");
+  spk_status st = make_map(qmap, q, s->head_dim, g.rows, g.units);
+  if (st != SPK_OK) return st;
+  return make_map(kmap, k, s->head_dim, s->n_in, g.units);
+}
+
+spk_status speckv_row_lse(const spk_speckv_shape* s, const void* q, const void* k, float* lse2, void* stream) {
+  SpeckvGeom g;
+  spk_status st = check_speckv(s, g);
+  if (st != SPK_OK) return st;
+  if (lse2 == nullptr) return fail(SPK_ERR_ARG, "lse2 must be non-NULL");
+  CUtensorMap qmap, kmap;
+  if ((st = speckv_maps(s, q, k, g, &qmap, &kmap)) != SPK_OK) return st;
+  ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
+                              s->layers, 0);
+  p.lse2 = lse2;
+  st = run_lse(p, qmap, kmap, s->head_dim, static_cast<cudaStream_t>(stream));
+  return st == SPK_OK ? ok() : st;
+}
+
+spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k, float* scores,
+                        float* window_mass, void* ws, size_t ws_bytes, void* stream) {
+  SpeckvGeom g;
+  spk_status st = check_speckv(s, g);
+  if (st != SPK_OK) return st;
+  if (g.n_pre > 0 && scores == nullptr) return fail(SPK_ERR_ARG, "scores must be non-NULL when n_window < n_in");
+  const size_t need = speckv_workspace_size(s);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
+  const int n_cols = static_cast<int>(window_mass ? s->n_in : g.n_pre);
+  if (n_cols == 0) return ok();
+  CUtensorMap qmap, kmap;
+  if ((st = speckv_maps(s, q, k, g, &qmap, &kmap)) != SPK_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
+                              s->layers, 0);
+  p.lse2 = static_cast<float*>(ws);
+  if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
+  p.n_pre = static_cast<int>(g.n_pre);
+  p.n_cols = n_cols;
+  p.out0 = scores;
+  p.out1 = window_mass;
+  p.n_blocks = (n_cols + 255) / 256;
+  p.n_items = p.n_units * p.n_blocks;
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  cudaError_t e = launch_score(MODE_COLSUM, s->head_dim, kmap, qmap, p, grid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
+  return ok();
+}
+
+// ------------------------------------------------------------------ SpecPC
+static spk_status check_specpc(const spk_specpc_shape* s, SpeckvGeom& g) {
+  if (s == nullptr) return fail(SPK_ERR_ARG, "shape is NULL");
+  if (s->batch < 1 || s->layers < 1 || s->hq < 1 || s->hkv < 1 || s->n_in < 1 || s->n_rows < 1)
+    return fail(SPK_ERR_ARG, "batch, layers, hq, hkv, n_in and n_rows must be >= 1");
+  if (s->hq % s->hkv != 0) return fail(SPK_ERR_ARG, "hq (%d) must be a multiple of hkv (%d)", s->hq, s->hkv);
+  if (s->l_skip < 0 || s->l_skip >= s->layers) return fail(SPK_ERR_ARG, "need 0 <= l_skip < layers");
+  if (s->n_lookahead < 1) return fail(SPK_ERR_ARG, "n_lookahead must be >= 1");
+  if (static_cast<long long>(s->n_rows) > static_cast<long long>(s->n_in) + s->n_lookahead - 1)
+    return fail(SPK_ERR_ARG, "n_rows must be <= n_in + n_lookahead - 1");
+  if (!(s->scale > 0.f) || !std::isfinite(s->scale)) return fail(SPK_ERR_ARG, "scale must be finite and > 0");
+  if (s->head_dim != 64) return fail(SPK_ERR_UNSUPPORTED, "SpecPC supports head_dim 64 (got %d)", s->head_dim);
+  g.g = s->hq / s->hkv;
+  if (g.g > kGroupMax) return fail(SPK_ERR_UNSUPPORTED, "hq/hkv = %d exceeds %d", g.g, kGroupMax);
+  g.R = s->n_rows;
+  g.rows = static_cast<long long>(g.g) * g.R;
+  if (g.rows > kRowsMax)
+    return fail(SPK_ERR_UNSUPPORTED, "(hq/hkv) * n_rows = %lld exceeds %d", g.rows, kRowsMax);
+  g.units = static_cast<long long>(s->batch) * (s->layers - s->l_skip) * s->hkv;
+  if (static_cast<long long>(s->batch) * s->layers * s->hkv * 8 > 0x7fffffffLL)
+    return fail(SPK_ERR_UNSUPPORTED, "too many units");
+  g.n_pre = s->n_in;
+  return SPK_OK;
+}
+
+size_t specpc_workspace_size(const spk_specpc_shape* s) {
+  SpeckvGeom g;
+  if (check_specpc(s, g) != SPK_OK) return 0;
+  return round_up(static_cast<size_t>(g.units) * g.rows * sizeof(float), 256);
+}
+
+spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k, const float* w, float* scores,
+                        void* ws, size_t ws_bytes, void* stream) {
+  SpeckvGeom g;
+  spk_status st = check_specpc(s, g);
+  if (st != SPK_OK) return st;
+  if (q == nullptr || k == nullptr || w == nullptr || scores == nullptr)
+    return fail(SPK_ERR_ARG, "q, k, row_weights and scores must be non-NULL device pointers");
+  if (!aligned16(q) || !aligned16(k)) return fail(SPK_ERR_ARG, "q and k must be 16-byte aligned");
+  const size_t need = specpc_workspace_size(s);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  const long long all_units = static_cast<long long>(s->batch) * s->layers * s->hkv;
+  CUtensorMap qmap, kmap;
+  if ((st = make_map(&qmap, q, s->head_dim, g.rows, all_units)) != SPK_OK) return st;
+  if ((st = make_map(&kmap, k, s->head_dim, s->n_in, all_units)) != SPK_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int c0 = s->n_in + s->n_lookahead - s->n_rows;
+  ScoreParams p = base_params(s->head_dim, s->n_in, g, c0, s->scale, s->hkv, s->layers - s->l_skip, s->layers,
+                              s->l_skip);
+  p.lse2 = static_cast<float*>(ws);
+  p.row_weights = w;
+  if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
+  p.row_weights = nullptr;
+  p.n_pre = s->n_in;
+  p.n_cols = s->n_in;
+  p.out0 = scores;
+  p.n_blocks = (s->n_in + 255) / 256;
+  p.n_items = s->batch * p.n_blocks;
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  cudaError_t e = launch_score(MODE_COLSUM_PC, s->head_dim, kmap, qmap, p, grid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "SpecPC column-sum launch");
+  return ok();
+}
+
+// ------------------------------------------------------------------ selection
+size_t topk_workspace_size(int units, int n_cand) {
+  if (units < 0 || n_cand < 0) return 0;
+  return round_up(topk_ws_bytes(units, n_cand), 256);
+}
+
+spk_status topk_select(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail,
+                       int32_t* idx, float* pooled, void* ws, size_t ws_bytes, void* stream) {
+  if (units < 0 || n_cand < 0 || k < 0 || n_tail < 0) return fail(SPK_ERR_ARG, "negative size");
+  if (pool_kernel < 1 || (pool_kernel & 1) == 0) return fail(SPK_ERR_ARG, "pool_kernel must be odd and >= 1");
+  if (units == 0) return ok();
+  const long long out_len = static_cast<long long>(k < n_cand ? k : n_cand) + n_tail;
+  if (out_len > 0 && idx == nullptr) return fail(SPK_ERR_ARG, "idx must be non-NULL");
+  if (n_cand > 0 && scores == nullptr) return fail(SPK_ERR_ARG, "scores must be non-NULL");
+  const size_t need = topk_workspace_size(units, n_cand);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (static_cast<long long>(units) > 0x7fffffffLL / (out_len > 0 ? out_len : 1) && out_len > 0)
+    return fail(SPK_ERR_UNSUPPORTED, "output too large");
+  cudaError_t e = launch_topk(scores, units, n_cand, pool_kernel, k, n_tail, idx, pooled, ws,
+                              static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+  return ok();
+}
+
+// ------------------------------------------------------------------ compaction
+spk_status kv_compact(const void* k, const void* v, int units, int n_src, int head_dim, int elem_bytes,
+                      const int32_t* idx, int n_idx, int units_per_idx, void* k_out, void* v_out, void* stream) {
+  if (units < 0 || n_src < 0 || n_idx < 0 || head_dim < 1 || elem_bytes < 1 || units_per_idx < 1)
+    return fail(SPK_ERR_ARG, "invalid sizes");
+  if (units % units_per_idx != 0) return fail(SPK_ERR_ARG, "units must be a multiple of units_per_idx");
+  const long long row_bytes = static_cast<long long>(head_dim) * elem_bytes;
+  if (row_bytes % 16 != 0) return fail(SPK_ERR_UNSUPPORTED, "head_dim * elem_bytes must be a multiple of 16");
+  if (units == 0 || n_idx == 0) return ok();
+  if (k == nullptr || k_out == nullptr || idx == nullptr) return fail(SPK_ERR_ARG, "k, k_out, idx must be non-NULL");
+  if ((v == nullptr) != (v_out == nullptr)) return fail(SPK_ERR_ARG, "v and v_out must both be set or both NULL");
+  if (!aligned16(k) || !aligned16(k_out) || (v && (!aligned16(v) || !aligned16(v_out))))
+    return fail(SPK_ERR_ARG, "k, v, k_out, v_out must be 16-byte aligned");
+  cudaError_t e = launch_compact(k, v, units, n_src, static_cast<int>(row_bytes), idx, n_idx, units_per_idx, k_out,
+                                 v_out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "compaction launch");
+  return ok();
+}
+
+// ------------------------------------------------------------------ device errors
+spk_status spk_device_error(int* status, int* site, int clear) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  int code = 0, where = 0;
+  if ((e = cudaMemcpyFromSymbol(&code, g_device_error, sizeof code)) != cudaSuccess)
+    return cuda_fail(e, "reading the device error word");
+  if ((e = cudaMemcpyFromSymbol(&where, g_device_error_site, sizeof where)) != cudaSuccess)
+    return cuda_fail(e, "reading the device error site");
+  if (clear) {
+    const int zero = 0;
+    if ((e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero)) != cudaSuccess)
+      return cuda_fail(e, "clearing the device error word");
+    if ((e = cudaMemcpyToSymbol(g_device_error_site, &zero, sizeof zero)) != cudaSuccess)
+      return cuda_fail(e, "clearing the device error site");
+  }
+  if (status) *status = code == SPK_DEVERR_NONE ? SPK_OK : (code == SPK_DEVERR_TIMEOUT ? SPK_ERR_TIMEOUT : SPK_ERR_ARG);
+  if (site) *site = where;
+  return ok();
+}
+
+}  // extern "C"
+
+namespace spk {
+namespace {
+// One thread waits on a barrier that nothing will ever complete; the bounded
+// wait gives up after limit_ns, records the timeout and returns.
+__global__ void wait_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, reinterpret_cast<volatile int*>(&abort_flag), 999, limit_ns);
+  }
+}
+}  // namespace
+}  // namespace spk
+
+extern "C" spk_status spk_selftest_wait_timeout(long long limit_ns, void* stream) {
+  if (limit_ns < 1000) limit_ns = 1000;
+  if (limit_ns > 1000000000LL) limit_ns = 1000000000LL;
+  spk::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_ns));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return spk::cuda_fail(e, "self-test launch");
+  return spk::ok();
+}

@@ -1,0 +1,58 @@
+// score.cuh -- parameters shared by the scoring kernel and its host launcher.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace spk {
+
+enum ScoreMode : int {
+  MODE_LSE = 0,        // pass 1: per query row, lse2 = log2 sum_j 2^(c2 q.k_j) over visible keys
+  MODE_COLSUM = 1,     // pass 2, SpecKV: per key, sum over the unit's rows of 2^(c2 q.k - lse2)
+  MODE_COLSUM_PC = 2,  // pass 2, SpecPC: per key, weighted layer/row mean per query head, max over heads
+};
+
+constexpr int kRowsMax = 2048;   // query rows per unit (g * rows-per-head) held in shared memory
+constexpr int kGroupMax = 16;    // SpecPC: query heads per KV head
+
+struct ScoreParams {
+  // geometry of a unit (one batch element, layer >= l_skip, KV head)
+  int head_dim;
+  int n_in;          // input keys per unit
+  int rows;          // query rows per unit = g * R, ordered [query head][row]
+  int R;             // rows per query head
+  int c0;            // head-local row i sees keys [0, min(n_in, c0 + i))
+  float c2;          // scale * log2(e)
+  // unit u = (b * layers_used + l') * hkv + h  ->  tensor coordinate
+  // (b * layers_total + l_skip + l') * hkv + h of the [B*L*Hkv][rows|n_in][d] views
+  int hkv;
+  int layers_used;
+  int layers_total;
+  int l_skip;
+  int n_units;
+  // work decomposition
+  int n_items;       // persistent-loop items
+  int n_blocks;      // items per unit (LSE: 256-row blocks) or per batch/unit (256-key blocks)
+  // buffers
+  float* lse2;       // [n_units][rows]: LSE writes it, the column passes read it
+  float* out0;       // SpecKV scores [n_units][n_pre] or SpecPC scores [batch][n_in]
+  float* out1;       // SpecKV window mass [n_units][n_in - n_pre] (nullable)
+  int n_pre;         // prefix keys that are scored
+  int n_cols;        // keys whose column sums are written
+  const float* row_weights;  // SpecPC row weights [R] (LSE folds -log2(w_i / norm) into lse2)
+};
+
+cudaError_t launch_score(int mode, int head_dim, const CUtensorMap& amap, const CUtensorMap& bmap,
+                         const ScoreParams& p, int grid, cudaStream_t stream);
+int score_smem_bytes(int mode, int head_dim);
+
+// pooling + top-k selection (select.cu)
+cudaError_t launch_topk(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail,
+                        int* idx, float* pooled, void* ws, cudaStream_t stream);
+size_t topk_ws_bytes(int units, int n_cand);
+
+// row gather (compact.cu)
+cudaError_t launch_compact(const void* k, const void* v, int units, int n_src, int row_bytes, const int* idx,
+                           int n_idx, int units_per_idx, void* k_out, void* v_out, cudaStream_t stream);
+
+}  // namespace spk

@@ -1,0 +1,221 @@
+"""GPU parity of the SpecKV path (scores -> pool + top-k + window -> compaction)
+against the fp64 oracle, through the C ABI (prompt_compression_b200.binding).
+
+Small cases run the oracle on every unit: they span several 128-key and
+128-row tiles, ragged tails, GQA groups, and the degenerate settings of the
+method (no lookahead = SnapKV-style scoring, no window, window = whole input,
+C_max >= n_pre).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from tests.gpu_helpers import (assert_indices_match, assert_scores_close, bits_of, oracle_unit,
+                               to_bf16_tensor)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def P():
+    import torch  # noqa: F401
+    from prompt_compression_b200 import build
+    build.build_library()
+    import prompt_compression_b200 as P
+    P.load_library()
+    P.spk_device_error(clear=True)
+    return P
+
+
+def _random_case(seed, B, L, hq, hkv, d, n_in, n_window, n_lookahead, planted=True):
+    rng = np.random.default_rng(seed)
+    R = n_window + n_lookahead
+    q = rng.standard_normal((B, L, hq, R, d)).astype(np.float32)
+    k = rng.standard_normal((B, L, hkv, n_in, d)).astype(np.float32)
+    v = rng.standard_normal((B, L, hkv, n_in, d)).astype(np.float32)
+    if planted:
+        u = rng.standard_normal((B, L, hkv, d)).astype(np.float32)
+        u /= np.linalg.norm(u, axis=-1, keepdims=True)
+        k[:, :, :, 0] += 4 * u
+        heavy = rng.choice(np.arange(1, max(n_in - n_window, 2)), size=max(1, n_in // 50), replace=False)
+        k[:, :, :, heavy] += 3 * u[:, :, :, None, :]
+        q += 1.5 * np.repeat(u, hq // hkv, axis=2)[:, :, :, None, :]
+    q /= math.sqrt(d)
+    return W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v)
+
+
+def _run_and_check(P, qb, kb, vb, n_window, c_max, pool=7, scale=1.0):
+    import torch
+    B, L, hq, R, d = qb.shape
+    hkv, n_in = kb.shape[2], kb.shape[3]
+    g = hq // hkv
+    n_lookahead = R - n_window
+    q, k, v = to_bf16_tensor(qb), to_bf16_tensor(kb), to_bf16_tensor(vb)
+    buf = P.pipeline.SpeckvBuffers(q, k, v, n_window, c_max, window_mass=n_window > 0, with_pooled=True)
+    P.speckv_compress(q, k, v, n_window, c_max, pool, scale, buffers=buf)
+    lse2 = torch.empty((buf.units, g * R), dtype=torch.float32, device="cuda")
+    P.speckv_row_lse(q, k, n_window, lse2, scale)
+    torch.cuda.synchronize()
+    assert P.spk_device_error() == (0, 0)
+    scores = buf.scores.cpu().numpy()
+    pooled = buf.pooled.cpu().numpy()
+    wmass = buf.window_mass.cpu().numpy() if buf.window_mass is not None else None
+    idx = buf.idx.cpu().numpy()
+    lse = lse2.cpu().numpy()
+    k_out, v_out = bits_of(buf.k_out), bits_of(buf.v_out)
+    n_pre = n_in - n_window
+    c = min(c_max, n_pre)
+    for u in range(buf.units):
+        b, l, h = u // (L * hkv), (u // hkv) % L, u % hkv
+        qu = qb[b, l, h * g:(h + 1) * g]
+        ku = kb[b, l, h]
+        s, wm, p, ridx = oracle_unit(qu, ku, n_window, n_lookahead, c_max, pool, scale)
+        _, _, olse = oracle.speckv_unit(qu, ku, n_window, n_lookahead, scale, with_lse=True)
+        # pass 1: log2-domain LSE of every row
+        np.testing.assert_allclose(lse[u], olse / math.log(2.0), rtol=0, atol=2e-5)
+        assert_scores_close(scores[u], s, f"scores[{u}]")
+        if wmass is not None:
+            assert_scores_close(wmass[u], wm, f"window_mass[{u}]")
+            # every row's softmax sums to 1: columns sum to g * R
+            tot = scores[u].astype(np.float64).sum() + wmass[u].astype(np.float64).sum()
+            assert abs(tot - g * R) < 1e-4 * g * R
+        # pooling is exact; selection is bit-exact on the GPU's own scores
+        np.testing.assert_array_equal(pooled[u], oracle.maxpool(scores[u].astype(np.float64), pool)
+                                      .astype(np.float32))
+        own = oracle.topk_with_tail(scores[u].astype(np.float64) if pool == 1 else
+                                    oracle.maxpool(scores[u].astype(np.float64), pool), c_max, n_window)
+        assert np.array_equal(idx[u], own), f"unit {u}: selection differs from the oracle on the same scores"
+        assert_indices_match(idx[u], ridx, p, c)
+        # compaction: bit-exact rows at the GPU's indices
+        np.testing.assert_array_equal(k_out[b, l, h], kb[b, l, h][idx[u]])
+        np.testing.assert_array_equal(v_out[b, l, h], vb[b, l, h][idx[u]])
+    return buf
+
+
+def test_tiny_workload(P):
+    q, k, v = W.tiny_speckv_numpy(0)
+    cfg = W.TINY
+    buf = _run_and_check(P, W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v), cfg.n_window, cfg.c_max, cfg.pool)
+    idx = buf.idx.cpu().numpy()
+    for u in range(buf.units):
+        assert {0, 100, 101, 102, 103} <= set(idx[u].tolist())
+
+
+@pytest.mark.parametrize("case", [
+    # seed, B, L, hq, hkv, d, n_in, n_window, n_lookahead, c_max
+    (1, 1, 2, 6, 2, 128, 1000, 40, 24, 100),     # ragged key tail, g=3, 192 rows
+    (2, 2, 1, 10, 2, 128, 700, 64, 32, 64),      # 480 rows: two row blocks, half-empty tile
+    (3, 1, 1, 4, 4, 64, 300, 0, 16, 32),         # no window
+    (4, 1, 1, 8, 2, 64, 513, 32, 0, 128),        # no lookahead (SnapKV-style)
+    (5, 1, 1, 2, 1, 128, 129, 16, 8, 500),       # C_max >= n_pre keeps everything
+    (6, 1, 1, 4, 2, 64, 96, 96, 4, 8),           # window covers the whole input
+    (7, 1, 3, 5, 1, 128, 2100, 64, 128, 256),    # Qwen-like group: 960 rows, 7.5 row tiles
+])
+def test_speckv_shapes(P, case):
+    seed, B, L, hq, hkv, d, n_in, nw, nl, c_max = case
+    qb, kb, vb = _random_case(seed, B, L, hq, hkv, d, n_in, nw, nl)
+    _run_and_check(P, qb, kb, vb, nw, c_max)
+
+
+def test_scale_argument(P):
+    qb, kb, vb = _random_case(11, 1, 1, 4, 2, 64, 400, 16, 16)
+    _run_and_check(P, qb, kb, vb, 16, 64, scale=0.61)
+
+
+def test_pool_kernel_one_and_three(P):
+    qb, kb, vb = _random_case(12, 1, 1, 4, 2, 64, 333, 8, 8)
+    _run_and_check(P, qb, kb, vb, 8, 40, pool=1)
+    _run_and_check(P, qb, kb, vb, 8, 40, pool=3)
+
+
+def test_deterministic(P):
+    import torch
+    qb, kb, vb = _random_case(13, 1, 2, 8, 2, 128, 1500, 32, 32)
+    q, k, v = to_bf16_tensor(qb), to_bf16_tensor(kb), to_bf16_tensor(vb)
+    a = P.speckv_compress(q, k, v, 32, 128, 7, window_mass=True)
+    sa, ia, ka = a.scores.clone(), a.idx.clone(), a.k_out.clone()
+    b = P.speckv_compress(q, k, v, 32, 128, 7, window_mass=True)
+    torch.cuda.synchronize()
+    assert torch.equal(sa, b.scores) and torch.equal(ia, b.idx) and torch.equal(ka, b.k_out)
+
+
+def test_uniform_keys_ties_lowest_index(P):
+    # identical keys: all prefix scores tie exactly -> indices 0..C-1
+    import torch
+    rng = np.random.default_rng(14)
+    d, n_in, nw, nl = 64, 640, 16, 16
+    q = (rng.standard_normal((1, 1, 4, nw + nl, d)) / 8).astype(np.float32)
+    k = np.tile(rng.standard_normal((1, 1, 2, 1, d)).astype(np.float32), (1, 1, 1, n_in, 1))
+    qb, kb = W.bf16_bits(q), W.bf16_bits(k)
+    buf = P.speckv_compress(to_bf16_tensor(qb), to_bf16_tensor(kb), to_bf16_tensor(kb), nw, 64, 7)
+    torch.cuda.synchronize()
+    idx = buf.idx.cpu().numpy()
+    for u in range(2):
+        assert idx[u].tolist() == list(range(64)) + list(range(n_in - nw, n_in))
+
+
+def test_topk_select_direct(P):
+    """topk_select alone on integer-valued scores (many exact ties), bit-exact."""
+    import torch
+    rng = np.random.default_rng(15)
+    for n, kk, tail, pool in [(5000, 300, 7, 7), (65472, 256, 64, 7), (100, 0, 5, 3), (37, 50, 0, 1),
+                              (2, 1, 0, 7), (0, 4, 3, 7)]:
+        s = rng.integers(0, 20, size=(3, n)).astype(np.float32) * 0.25
+        st = torch.from_numpy(s).cuda()
+        c = min(kk, n)
+        idx = torch.empty((3, c + tail), dtype=torch.int32, device="cuda")
+        P.topk_select(st, kk, tail, idx, pool)
+        torch.cuda.synchronize()
+        got = idx.cpu().numpy()
+        for u in range(3):
+            ref = oracle.topk_with_tail(oracle.maxpool(s[u].astype(np.float64), pool) if n else
+                                        np.zeros(0), kk, tail)
+            assert got[u].tolist() == ref.tolist(), (n, kk, tail, pool)
+
+
+def test_kv_compact_broadcast_and_errors(P):
+    import torch
+    rng = np.random.default_rng(16)
+    units, n_src, d = 6, 300, 64
+    kb = rng.integers(0, 2 ** 16, size=(units, n_src, d), dtype=np.uint16)
+    vb = rng.integers(0, 2 ** 16, size=(units, n_src, d), dtype=np.uint16)
+    idx = np.stack([np.sort(rng.choice(n_src, 40, replace=False)) for _ in range(2)]).astype(np.int32)
+    k, v = to_bf16_tensor(kb), to_bf16_tensor(vb)
+    ko = torch.empty((units, 40, d), dtype=torch.bfloat16, device="cuda")
+    vo = torch.empty_like(ko)
+    P.kv_compact(k, v, torch.from_numpy(idx).cuda(), ko, vo, units_per_idx=3)
+    torch.cuda.synchronize()
+    ko_b, vo_b = bits_of(ko), bits_of(vo)
+    for u in range(units):
+        np.testing.assert_array_equal(ko_b[u], kb[u][idx[u // 3]])
+        np.testing.assert_array_equal(vo_b[u], vb[u][idx[u // 3]])
+    assert P.spk_device_error() == (0, 0)
+    bad = idx.copy()
+    bad[1, 5] = n_src     # out of range: recorded, row left unwritten, nothing faults
+    P.kv_compact(k, v, torch.from_numpy(bad).cuda(), ko, vo, units_per_idx=3)
+    st, site = P.spk_device_error()
+    assert st == P.binding.SPK_ERR_ARG
+    assert P.spk_device_error() == (0, 0)
+
+
+def test_argument_errors_do_not_launch(P):
+    import torch
+    q = torch.zeros((1, 1, 4, 8, 96), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((1, 1, 2, 64, 96), dtype=torch.bfloat16, device="cuda")
+    s = torch.zeros((2, 60), dtype=torch.float32, device="cuda")
+    with pytest.raises(P.SpeckvError) as e:
+        P.speckv_score(q, k, 4, s)
+    assert e.value.status == P.binding.SPK_ERR_UNSUPPORTED
+    q = torch.zeros((1, 1, 4, 8, 64), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((1, 1, 3, 64, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(P.SpeckvError) as e:
+        P.speckv_score(q, k, 4, s)
+    assert e.value.status == P.binding.SPK_ERR_ARG
+    k = torch.zeros((1, 1, 2, 64, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(P.SpeckvError) as e:
+        P.speckv_score(q, k, 4, s, workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == P.binding.SPK_ERR_WORKSPACE
+    assert P.spk_device_error() == (0, 0)

@@ -313,3 +313,21 @@ def specpc_inputs(cfg: SpecPCConfig, seed: int = 0, device="cpu", heavy_pos=None
         q[:, l].copy_(ql)
         del kl, ql
     return {"q": q, "k": k, "heavy": heavy}
+
+
+def speckv_unit_numpy(cfg: SpecKVConfig, seed: int, unit: int):
+    """One unit's inputs (bf16 bit patterns) drawn on the host with numpy:
+    q [g, R, d], k [n_in, d], v [n_in, d], same distribution as speckv_inputs
+    (sink, heavy keys with the clustered layout of the config, query offset)."""
+    rng = np.random.default_rng([seed, unit])
+    d, g = cfg.head_dim, cfg.g
+    q = rng.standard_normal((g, cfg.rows, d)).astype(np.float32)
+    k = rng.standard_normal((cfg.n_in, d)).astype(np.float32)
+    v = rng.standard_normal((cfg.n_in, d)).astype(np.float32)
+    u = _unit(rng.standard_normal(d)).astype(np.float32)
+    hp = heavy_positions(max(cfg.n_pre, 2), cfg.heavy_frac, cfg.heavy_spans, cfg.span_len, seed * 1000)
+    k[0] += cfg.sink * u
+    k[hp] += cfg.heavy * u
+    q += cfg.q_offset * u
+    q *= np.float32(1.0 / math.sqrt(d))
+    return bf16_bits(q), bf16_bits(k), bf16_bits(v)
