@@ -93,6 +93,24 @@ spk_status speckv_score(const spk_speckv_shape* shape, const void* q_bf16, const
 spk_status speckv_row_lse(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16,
                           float* lse2, void* stream);
 
+/* speckv_score for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this is a deployment variant.  Serving engines that
+ * reserve nearly all of HBM for their own KV-cache pool, and plugin hosts
+ * that give plugins no access to the CUDA allocator, can neither cudaMalloc
+ * nor spare a workspace; this call keeps pass 1's row-LSE scratch in a fixed
+ * 4 MiB array inside the library image instead (no allocation of any kind).
+ *   - Same shapes, layouts, outputs and rules as speckv_score.
+ *   - Rejects (SPK_ERR_UNSUPPORTED, before any launch) shapes needing more
+ *     than 1,048,576 floats of scratch: units * (hq/hkv) * (n_window + n_lookahead).
+ *   - Every GPU that loads the library holds the 4 MiB until process exit.
+ *   - The first call on a device looks up the array's address on that device
+ *     (cudaGetSymbolAddress) and caches it: make it before any stream capture.
+ *   - All calls share the array, which keeps the last call's contents (every
+ *     entry read is first rewritten by the same call, so nothing needs
+ *     clearing); calls whose kernels overlap on the GPU race on it. */
+spk_status speckv_score_static_ws(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16,
+                                  float* scores, float* window_mass, void* stream);
+
 /* ------------------------------------------------------------------------
  * SpecPC scoring (section 关键设计, SpecPC)
  *

@@ -364,3 +364,92 @@ extern "C" spk_status spk_selftest_wait_timeout(long long limit_ns, void* stream
   if (e != cudaSuccess) return spk::cuda_fail(e, "self-test launch");
   return spk::ok();
 }
+
+// ---------------------------------------------------------------------------
+// speckv_score_static_ws: speckv_score without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory on this path: serving engines
+// that reserve nearly all of HBM up front for their KV-cache pool and hand
+// memory out only through their own allocator, and plugin hosts that give a
+// plugin no access to the CUDA allocator.  They also cannot always find room
+// for a workspace.  This entry point keeps the row-LSE scratch of pass 1 in a
+// fixed array that lives in the library image itself, so a call allocates
+// nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+//
+// Limits and behaviour:
+//   - the scratch holds kStaticLseFloats = 1,048,576 floats (4 MiB); a shape
+//     with units * (hq/hkv) * (n_window + n_lookahead) above that is rejected
+//     with SPK_ERR_UNSUPPORTED before anything is launched;
+//   - every GPU that loads the library keeps these 4 MiB until the process exits;
+//   - the first call on each device looks up the array's device address with
+//     that device current (cudaGetSymbolAddress) and caches it; make that
+//     first call before any stream capture;
+//   - all calls share the one array and it keeps the previous call's contents.
+//     Pass 1 overwrites every entry pass 2 reads, so nothing has to start at
+//     zero, but calls whose kernels overlap on the GPU (different streams
+//     without ordering between them) race on the array: order them.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace spk {
+namespace {
+constexpr long long kStaticLseFloats = 1LL << 20;
+constexpr int kMaxDevices = 64;
+static __device__ __align__(256) float g_static_lse2[kStaticLseFloats];
+float* g_static_lse2_addr[kMaxDevices] = {};
+std::mutex g_static_lse2_mu;
+
+// Device address of g_static_lse2 on the current device (looked up once per device).
+spk_status static_lse2_address(float** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SPK_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_static_lse2_mu);
+  if (g_static_lse2_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_lse2);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+    g_static_lse2_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_static_lse2_addr[dev];
+  return SPK_OK;
+}
+}  // namespace
+}  // namespace spk
+
+extern "C" spk_status speckv_score_static_ws(const spk_speckv_shape* s, const void* q, const void* k,
+                                             float* scores, float* window_mass, void* stream) {
+  using namespace spk;
+  SpeckvGeom g;
+  spk_status st = check_speckv(s, g);
+  if (st != SPK_OK) return st;
+  const long long need = g.units * g.rows;
+  if (need > kStaticLseFloats)
+    return fail(SPK_ERR_UNSUPPORTED,
+                "units * (hq/hkv) * (n_window + n_lookahead) = %lld exceeds the static scratch of %lld floats; "
+                "use speckv_score with a workspace",
+                need, kStaticLseFloats);
+  if (g.n_pre > 0 && scores == nullptr) return fail(SPK_ERR_ARG, "scores must be non-NULL when n_window < n_in");
+  const int n_cols = static_cast<int>(window_mass ? s->n_in : g.n_pre);
+  if (n_cols == 0) return ok();
+  CUtensorMap qmap, kmap;
+  if ((st = speckv_maps(s, q, k, g, &qmap, &kmap)) != SPK_OK) return st;
+  float* lse2 = nullptr;
+  if ((st = static_lse2_address(&lse2)) != SPK_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
+                              s->layers, 0);
+  p.lse2 = lse2;
+  if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
+  p.n_pre = static_cast<int>(g.n_pre);
+  p.n_cols = n_cols;
+  p.out0 = scores;
+  p.out1 = window_mass;
+  p.n_blocks = (n_cols + 255) / 256;
+  p.n_items = p.n_units * p.n_blocks;
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  cudaError_t e = launch_score(MODE_COLSUM, s->head_dim, kmap, qmap, p, grid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
+  return ok();
+}
