@@ -196,6 +196,12 @@ const char* spk_last_error(void);
  * device could not be read. */
 spk_status spk_device_error(int* status, int* site, int clear);
 
+/* Diagnostic: y[i] = 2^t[i] as computed on the FMA pipe by the scoring
+ * epilogues (range reduction + fitted degree-5 polynomial, relative error
+ * <= 2.2e-7 for t in [-126, 64); arguments below -126 give a value under
+ * 1.2e-38).  t, y: fp32 device arrays of n elements. */
+spk_status spk_exp2_fma(const float* t, float* y, int n, void* stream);
+
 /* Self-test of the bounded waits: launches one kernel that waits on a barrier
  * nothing will complete, with a limit of limit_ns nanoseconds (clamped to
  * [1e3, 1e9]).  The kernel gives up, records SPK_ERR_TIMEOUT at site 999 and

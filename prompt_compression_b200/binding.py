@@ -68,6 +68,7 @@ def load_library():
         "spk_last_error": (ctypes.c_char_p, []),
         "spk_device_error": (I, [ctypes.POINTER(I), ctypes.POINTER(I), I]),
         "spk_selftest_wait_timeout": (I, [ctypes.c_longlong, vp]),
+        "spk_exp2_fma": (I, [vp, vp, I, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -211,3 +212,10 @@ def spk_device_error(clear: bool = True):
 
 def spk_selftest_wait_timeout(limit_ns: int, stream=None):
     _check(load_library().spk_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def spk_exp2_fma(t, y, stream=None):
+    """y = 2^t through the scoring epilogues' FMA-pipe exponential (diagnostic)."""
+    _check(load_library().spk_exp2_fma(_dev(t, "t", torch.float32), _dev(y, "y", torch.float32), t.numel(),
+                                       _stream(stream)))
+    return y

@@ -11,6 +11,7 @@
 
 #include "../../include/speckv.h"
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "score.cuh"
 
 namespace spk {
@@ -146,10 +147,13 @@ extern "C" {
 
 const char* spk_last_error(void) { return g_msg; }
 
+// Row offsets between the passes: [units][rows rounded up to 128] floats.
+static long long rows_padded(long long rows) { return (rows + 127) / 128 * 128; }
+
 size_t speckv_workspace_size(const spk_speckv_shape* s) {
   SpeckvGeom g;
   if (check_speckv(s, g) != SPK_OK) return 0;
-  return round_up(static_cast<size_t>(g.units) * g.rows * sizeof(float), 256);
+  return round_up(static_cast<size_t>(g.units) * rows_padded(g.rows) * sizeof(float), 256);
 }
 
 static spk_status speckv_maps(const spk_speckv_shape* s, const void* q, const void* k, const SpeckvGeom& g,
@@ -171,6 +175,8 @@ spk_status speckv_row_lse(const spk_speckv_shape* s, const void* q, const void* 
   ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
                               s->layers, 0);
   p.lse2 = lse2;
+  p.lse_stride = static_cast<int>(g.rows);
+  p.lse_store = 0;
   st = run_lse(p, qmap, kmap, s->head_dim, static_cast<cudaStream_t>(stream));
   return st == SPK_OK ? ok() : st;
 }
@@ -193,6 +199,8 @@ spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k,
   ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
                               s->layers, 0);
   p.lse2 = static_cast<float*>(ws);
+  p.lse_stride = static_cast<int>(rows_padded(g.rows));
+  p.lse_store = 1;
   if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
   p.n_pre = static_cast<int>(g.n_pre);
   p.n_cols = n_cols;
@@ -219,7 +227,7 @@ static spk_status check_specpc(const spk_specpc_shape* s, SpeckvGeom& g) {
   if (!(s->scale > 0.f) || !std::isfinite(s->scale)) return fail(SPK_ERR_ARG, "scale must be finite and > 0");
   if (s->head_dim != 64) return fail(SPK_ERR_UNSUPPORTED, "SpecPC supports head_dim 64 (got %d)", s->head_dim);
   g.g = s->hq / s->hkv;
-  if (g.g > kGroupMax) return fail(SPK_ERR_UNSUPPORTED, "hq/hkv = %d exceeds %d", g.g, kGroupMax);
+  if (s->hq > kHeadsMax) return fail(SPK_ERR_UNSUPPORTED, "hq = %d exceeds %d", s->hq, kHeadsMax);
   g.R = s->n_rows;
   g.rows = static_cast<long long>(g.g) * g.R;
   if (g.rows > kRowsMax)
@@ -234,7 +242,7 @@ static spk_status check_specpc(const spk_specpc_shape* s, SpeckvGeom& g) {
 size_t specpc_workspace_size(const spk_specpc_shape* s) {
   SpeckvGeom g;
   if (check_specpc(s, g) != SPK_OK) return 0;
-  return round_up(static_cast<size_t>(g.units) * g.rows * sizeof(float), 256);
+  return round_up(static_cast<size_t>(g.units) * rows_padded(g.rows) * sizeof(float), 256);
 }
 
 spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k, const float* w, float* scores,
@@ -248,6 +256,7 @@ spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k,
   const size_t need = specpc_workspace_size(s);
   if (ws == nullptr || ws_bytes < need)
     return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
   const long long all_units = static_cast<long long>(s->batch) * s->layers * s->hkv;
   CUtensorMap qmap, kmap;
   if ((st = make_map(&qmap, q, s->head_dim, g.rows, all_units)) != SPK_OK) return st;
@@ -257,6 +266,8 @@ spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k,
   ScoreParams p = base_params(s->head_dim, s->n_in, g, c0, s->scale, s->hkv, s->layers - s->l_skip, s->layers,
                               s->l_skip);
   p.lse2 = static_cast<float*>(ws);
+  p.lse_stride = static_cast<int>(rows_padded(g.rows));
+  p.lse_store = 1;
   p.row_weights = w;
   if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
   p.row_weights = nullptr;
@@ -424,10 +435,11 @@ extern "C" spk_status speckv_score_static_ws(const spk_speckv_shape* s, const vo
   SpeckvGeom g;
   spk_status st = check_speckv(s, g);
   if (st != SPK_OK) return st;
-  const long long need = g.units * g.rows;
+  const long long need = g.units * rows_padded(g.rows);
   if (need > kStaticLseFloats)
     return fail(SPK_ERR_UNSUPPORTED,
-                "units * (hq/hkv) * (n_window + n_lookahead) = %lld exceeds the static scratch of %lld floats; "
+                "units * (hq/hkv) * (n_window + n_lookahead), rows rounded up to 128, = %lld exceeds the static "
+                "scratch of %lld floats; "
                 "use speckv_score with a workspace",
                 need, kStaticLseFloats);
   if (g.n_pre > 0 && scores == nullptr) return fail(SPK_ERR_ARG, "scores must be non-NULL when n_window < n_in");
@@ -441,6 +453,8 @@ extern "C" spk_status speckv_score_static_ws(const spk_speckv_shape* s, const vo
   ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
                               s->layers, 0);
   p.lse2 = lse2;
+  p.lse_stride = static_cast<int>(rows_padded(g.rows));
+  p.lse_store = 1;
   if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
   p.n_pre = static_cast<int>(g.n_pre);
   p.n_cols = n_cols;
@@ -452,4 +466,34 @@ extern "C" spk_status speckv_score_static_ws(const spk_speckv_shape* s, const vo
   cudaError_t e = launch_score(MODE_COLSUM, s->head_dim, kmap, qmap, p, grid, cs);
   if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
   return ok();
+}
+
+// ---------------------------------------------------------------------------
+// spk_exp2_fma: the FMA-pipe exponential of the scoring epilogues, exposed
+// so that tests can compare it with exp2 over its whole argument range.
+// ---------------------------------------------------------------------------
+namespace spk {
+namespace {
+__global__ void exp2_fma_kernel(const float* __restrict__ t, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_fma_pair(f2(t[i], t[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_fma_pair(f2(t[i], t[i])).x;
+  }
+}
+}  // namespace
+}  // namespace spk
+
+extern "C" spk_status spk_exp2_fma(const float* t, float* y, int n, void* stream) {
+  if (n < 0) return spk::fail(SPK_ERR_ARG, "n must be >= 0");
+  if (n == 0) return spk::ok();
+  if (t == nullptr || y == nullptr) return spk::fail(SPK_ERR_ARG, "t and y must be non-NULL device pointers");
+  const int pairs = (n + 1) / 2;
+  spk::exp2_fma_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(t, y, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return spk::cuda_fail(e, "exp2 launch");
+  return spk::ok();
 }

@@ -17,13 +17,21 @@
 //   pass 2 (MODE_COLSUM / MODE_COLSUM_PC): lane = key, columns = query rows;
 //                      sum_rows 2^(c2 * q.k - lse2[row]) is the key's score.
 // Both passes share one persistent, warp-specialised kernel:
-//   warp 8   : TMA producer (A tiles once per segment, B tiles streamed)
-//   warp 9   : TMEM allocator + single-thread UMMA issuer (128 x N x 16 bf16)
-//   warps 0-7: epilogue; warpgroup t owns A tile t, each thread one TMEM lane.
+//   warp 16   : TMA producer: an item's two A tiles once per segment, the
+//               segment's row offsets (-lse2, one bulk copy), B tiles streamed
+//   warp 17   : TMEM allocator + single-thread UMMA issuer (128 x N x 16 bf16)
+//   warps 0-15: epilogue; warp w owns TMEM lane quadrant w % 4 of A tile w / 8
+//               and one 64-column half of every accumulator stage (four warps
+//               per SM sub-partition hide the latency of the exp2 chains); the
+//               two halves of a lane are merged in shared memory per item.
 // TMEM holds 2 accumulator stages x 2 A tiles x 128 fp32 columns (512 cols).
+// The epilogues work on 64 columns per TMEM wait with packed fp32x2 math;
+// 3 of every 8 exponential pairs run on the FMA pipe (exp2_poly.cuh), the
+// rest on the MUFU, so that neither unit alone bounds the pass.
 // No atomics: every output element is reduced by exactly one thread in a
 // fixed order, so results are bitwise reproducible.
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "score.cuh"
 
 namespace spk {
@@ -33,8 +41,13 @@ __device__ int g_device_error_site = 0;
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kEpiThreads = 256;
+// 16 epilogue warps (4 per SM sub-partition, to hide latency), then the
+// producer warp and the MMA warp.
+constexpr int kEpiWarps = 16;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 18 * 32;
 
 template <int MODE, int D>
 struct Cfg {
@@ -46,7 +59,7 @@ struct Cfg {
   static constexpr int kSmemA = kAStages * kABytes;
   static constexpr int kSmemB = kBStages * kTileBytes;
   static constexpr int kLseFloats = (MODE == MODE_LSE) ? 0 : 2 * kRowsMax;
-  static constexpr int kAccFloats = (MODE == MODE_COLSUM_PC) ? kGroupMax * 256 : 0;
+  static constexpr int kAccFloats = (MODE == MODE_COLSUM_PC) ? 2 * kHeadsMax * 256 : 0;
   static constexpr int kSmemBytes = 1024 + kSmemA + kSmemB + 4 * (kLseFloats + kAccFloats);
 };
 
@@ -94,61 +107,80 @@ __device__ __forceinline__ int chunk_cols(const ScoreParams& p, int bt) {
 }
 
 // ---------------------------------------------------------------------------
-// pass-1 epilogue: online log2-sum-exp2 over 32 keys of one row
+// pass-1 epilogue: online log2-sum-exp2 over 64 keys (jb .. jb+63) of one row
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void lse_update(const uint32_t (&v)[32], int jb, int c, float c2, float& m,
-                                           float& l) {
+__device__ __forceinline__ void lse_update64(const uint32_t (&va)[32], const uint32_t (&vb)[32], int jb, int c,
+                                             float c2, float& m, float& l) {
   if (jb >= c) return;
-  float x[32];
-  if (jb + 32 <= c) {
+  float x[64];
 #pragma unroll
-    for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(v[k]);
-  } else {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) x[k] = (jb + k < c) ? __uint_as_float(v[k]) : -INFINITY;
+  for (int k = 0; k < 32; ++k) {
+    x[k] = __uint_as_float(va[k]);
+    x[32 + k] = __uint_as_float(vb[k]);
   }
-  float mx = x[0];
+  if (jb + 64 > c) {
 #pragma unroll
-  for (int k = 1; k < 32; ++k) mx = fmaxf(mx, x[k]);
+    for (int k = 0; k < 64; ++k)
+      if (jb + k >= c) x[k] = -INFINITY;
+  }
+  float a0 = fmaxf(x[0], x[1]), a1 = fmaxf(x[2], x[3]), a2 = fmaxf(x[4], x[5]), a3 = fmaxf(x[6], x[7]);
+#pragma unroll
+  for (int k = 8; k < 64; k += 8) {
+    a0 = max3f(a0, x[k + 0], x[k + 1]);
+    a1 = max3f(a1, x[k + 2], x[k + 3]);
+    a2 = max3f(a2, x[k + 4], x[k + 5]);
+    a3 = max3f(a3, x[k + 6], x[k + 7]);
+  }
+  const float mx = max3f(a0, a1, fmaxf(a2, a3));
   const float mn = fmaxf(m, mx * c2);
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  const float2 c2v = f2(c2, c2), nm = f2(-mn, -mn);
+  float2 s[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-  for (int k = 0; k < 32; k += 4) {
-    s0 += ex2_approx(fmaf(x[k + 0], c2, -mn));
-    s1 += ex2_approx(fmaf(x[k + 1], c2, -mn));
-    s2 += ex2_approx(fmaf(x[k + 2], c2, -mn));
-    s3 += ex2_approx(fmaf(x[k + 3], c2, -mn));
+  for (int p = 0; p < 32; ++p) {
+    const float2 t = __ffma2_rn(f2(x[2 * p], x[2 * p + 1]), c2v, nm);
+    const float2 e = ((p & 7) < kPolyPairsOf8) ? exp2_fma_pair(t) : exp2_mufu_pair(t);
+    s[p & 3] = __fadd2_rn(s[p & 3], e);
   }
-  l = fmaf(l, ex2_approx(m - mn), (s0 + s1) + (s2 + s3));
+  const float2 s01 = __fadd2_rn(__fadd2_rn(s[0], s[1]), __fadd2_rn(s[2], s[3]));
+  if (mn > m) l *= ex2_approx(m - mn);    // first update: m = -inf, ex2(-inf) = 0
+  l += s01.x + s01.y;
   m = mn;
 }
 
 // ---------------------------------------------------------------------------
-// pass-2 epilogue: sum over 32 query rows nb..nb+31 of 2^(c2 x - off[row])
+// pass-2 epilogue: s += 2^(c2 x + off[row]) over 32 rows, off = -lse2
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float colsum32(const uint32_t (&v)[32], const float* off, int nb, float c2) {
-  const float4* o4 = reinterpret_cast<const float4*>(off + nb);
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+__device__ __forceinline__ void colsum32(const uint32_t (&v)[32], const float* off, float c2, float2 (&s)[4]) {
+  const float4* o4 = reinterpret_cast<const float4*>(off);
+  const float2 c2v = f2(c2, c2);
 #pragma unroll
-  for (int k = 0; k < 32; k += 4) {
-    const float4 o = o4[k / 4];
-    s0 += ex2_approx(fmaf(__uint_as_float(v[k + 0]), c2, -o.x));
-    s1 += ex2_approx(fmaf(__uint_as_float(v[k + 1]), c2, -o.y));
-    s2 += ex2_approx(fmaf(__uint_as_float(v[k + 2]), c2, -o.z));
-    s3 += ex2_approx(fmaf(__uint_as_float(v[k + 3]), c2, -o.w));
+  for (int q = 0; q < 8; ++q) {
+    const float4 o = o4[q];
+    const float2 t0 = __ffma2_rn(f2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), c2v, f2(o.x, o.y));
+    const float2 t1 =
+        __ffma2_rn(f2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), c2v, f2(o.z, o.w));
+    const int p0 = 2 * q, p1 = 2 * q + 1;
+    const float2 e0 = ((p0 & 7) < kPolyPairsOf8) ? exp2_fma_pair(t0) : exp2_mufu_pair(t0);
+    const float2 e1 = ((p1 & 7) < kPolyPairsOf8) ? exp2_fma_pair(t1) : exp2_mufu_pair(t1);
+    s[p0 & 3] = __fadd2_rn(s[p0 & 3], e0);
+    s[p1 & 3] = __fadd2_rn(s[p1 & 3], e1);
   }
-  return (s0 + s1) + (s2 + s3);
 }
 
-// Same, for a key j that some rows cannot see: row n (head-local i = n % R)
-// sees key j only if j < c0 + i.
+__device__ __forceinline__ float fold(const float2 (&s)[4]) {
+  const float2 t = __fadd2_rn(__fadd2_rn(s[0], s[1]), __fadd2_rn(s[2], s[3]));
+  return t.x + t.y;
+}
+
+// For a key j that some rows cannot see: row n (head-local i = n % R) sees
+// key j only if j < c0 + i.  nb is the first row of the 32.
 __device__ __forceinline__ float colsum32_masked(const uint32_t (&v)[32], const float* off, int nb, float c2,
                                                  int j, int c0, int R) {
   float s = 0.f;
   int i = nb % R;
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
-    if (j < c0 + i) s += ex2_approx(fmaf(__uint_as_float(v[k]), c2, -off[nb + k]));
+    if (j < c0 + i) s += ex2_approx(fmaf(__uint_as_float(v[k]), c2, off[k]));
     if (++i == R) i = 0;
   }
   return s;
@@ -156,6 +188,8 @@ __device__ __forceinline__ float colsum32_masked(const uint32_t (&v)[32], const 
 
 }  // namespace
 
+// 18 warps: two SM sub-partitions hold 5 warps, so at most 96 registers per
+// thread fit their 16,384-register files.
 template <int MODE, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
@@ -165,14 +199,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* const A_s = smem;
   uint8_t* const B_s = smem + C::kSmemA;
-  float* const lse_s = reinterpret_cast<float*>(B_s + C::kSmemB);
-  float* const acc_s = lse_s + C::kLseFloats;
+  float* const off_s = reinterpret_cast<float*>(B_s + C::kSmemB);   // 2 x kRowsMax row offsets
+  float* const acc_s = off_s + C::kLseFloats;                         // SpecPC: [2][kHeadsMax][256]
 
   __shared__ __align__(8) uint64_t a_full[2], a_empty[2], b_full[8], b_empty[8], acc_full[2], acc_empty[2],
-      off_ready[2], done_bar;
+      off_full[2], off_empty[2], mrg_full, mrg_empty, done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
   __shared__ float wsum_s[kThreads / 32];
+  __shared__ float xm_s[256], xl_s[256];   // column-half merge of per-row / per-key partials
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -180,17 +215,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kAStages; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], 1); }
     for (int s = 0; s < C::kBStages; ++s) { mbar_init(&b_full[s], 1); mbar_init(&b_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], 8); }
-    for (int s = 0; s < 2; ++s) mbar_init(&off_ready[s], kEpiThreads);
+    for (int s = 0; s < 2; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&off_full[s], 1); mbar_init(&off_empty[s], kEpiWarps); }
+    mbar_init(&mrg_full, kEpiWarps / 2);
+    mbar_init(&mrg_empty, kEpiWarps / 2);
     mbar_init(&done_bar, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&tmem_holder, 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_map(&amap);
     tma_prefetch_map(&bmap);
   }
@@ -218,15 +255,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nseg = n_segments(p, MODE);
   const int nb = b_tiles(p, MODE);
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t a_stage = 0, a_phase = 0, b_stage = 0, b_phase = 0;
       int a_last[2] = {-1, -1};
       int b_last[8] = {-1, -1, -1, -1, -1, -1, -1, -1};
+      int o_last[2] = {-1, -1};
+      int seg_count = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        for (int seg = 0; ok && seg < nseg; ++seg) {
+        for (int seg = 0; ok && seg < nseg; ++seg, ++seg_count) {
           int u, tc, a_row0;
           decode(p, MODE, item, seg, u, tc, a_row0);
           if (!(ok = mbar_wait(&a_empty[a_stage], a_phase ^ 1, abort_v, site(MODE, 0, 0)))) break;
@@ -240,6 +279,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                           tc);
           a_last[a_stage] = static_cast<int>(a_phase);
           if (++a_stage == C::kAStages) { a_stage = 0; a_phase ^= 1; }
+          if (MODE != MODE_LSE) {
+            // this segment's row offsets: -lse2 of unit u, padded with -inf
+            const int ob = seg_count & 1;
+            const uint32_t oph = (seg_count >> 1) & 1;
+            if (!(ok = mbar_wait(&off_empty[ob], oph ^ 1, abort_v, site(MODE, 0, 2)))) break;
+            const uint32_t bytes = static_cast<uint32_t>(p.lse_stride) * 4u;
+            mbar_arrive_expect_tx(&off_full[ob], bytes);
+            bulk_load(off_s + ob * kRowsMax, p.lse2 + static_cast<size_t>(u) * p.lse_stride, bytes, &off_full[ob]);
+            o_last[ob] = static_cast<int>(oph);
+          }
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = mbar_wait(&b_empty[b_stage], b_phase ^ 1, abort_v, site(MODE, 0, 1)))) break;
             mbar_arrive_expect_tx(&b_full[b_stage], C::kTileBytes);
@@ -257,12 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (these waits ignore the abort flag but are still time-bounded)
         volatile int never = 0;
         for (int s = 0; s < C::kAStages; ++s)
-          if (a_last[s] >= 0) mbar_wait(&a_full[s], a_last[s], &never, site(MODE, 0, 8), 100000000ull);
+          if (a_last[s] >= 0) mbar_wait(&a_full[s], a_last[s], &never, site(MODE, 0, 7), 100000000ull);
         for (int s = 0; s < C::kBStages; ++s)
-          if (b_last[s] >= 0) mbar_wait(&b_full[s], b_last[s], &never, site(MODE, 0, 9), 100000000ull);
+          if (b_last[s] >= 0) mbar_wait(&b_full[s], b_last[s], &never, site(MODE, 0, 8), 100000000ull);
+        for (int s = 0; s < 2; ++s)
+          if (o_last[s] >= 0) mbar_wait(&off_full[s], o_last[s], &never, site(MODE, 0, 9), 100000000ull);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       uint32_t a_stage = 0, a_phase = 0, b_stage = 0, b_phase = 0, acc_stage = 0, acc_phase = 0;
@@ -275,23 +326,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool act1 = a_tile_active(p, MODE, a_row0, 1);
           if (!(ok = mbar_wait(&a_full[a_stage], a_phase, abort_v, site(MODE, 1, 0)))) break;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(A_s + a_stage * C::kABytes);
+          const uint64_t a_desc0 = sw128_kmajor_desc(smem_u32(A_s + a_stage * C::kABytes));
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = mbar_wait(&b_full[b_stage], b_phase, abort_v, site(MODE, 1, 1)))) break;
             if (!(ok = mbar_wait(&acc_empty[acc_stage], acc_phase ^ 1, abort_v, site(MODE, 1, 2)))) break;
             tc_fence_after();
             const int n = (MODE == MODE_LSE) ? 128 : chunk_cols(p, bt);
             const uint32_t idesc = idesc_bf16_f32(128, n);
-            const uint32_t b_base = smem_u32(B_s + b_stage * C::kTileBytes);
+            const uint64_t b_desc0 = sw128_kmajor_desc(smem_u32(B_s + b_stage * C::kTileBytes));
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
               if (!(t == 0 ? act0 : act1)) continue;
               const uint32_t d_tmem = tmem_base + (acc_stage * 2 + t) * 128;
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                umma_bf16_ss(d_tmem, sw128_kmajor_desc(a_base + t * C::kTileBytes + koff),
-                             sw128_kmajor_desc(b_base + koff), idesc, kk > 0 ? 1u : 0u);
+                // descriptor start addresses advance in 16-byte units
+                const uint64_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                umma_bf16_ss(d_tmem, a_desc0 + ((t * C::kTileBytes) >> 4) + koff, b_desc0 + koff, idesc,
+                             kk > 0 ? 1u : 0u);
               }
             }
             umma_commit(&acc_full[acc_stage]);
@@ -311,176 +363,219 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int t = warp >> 2;             // A tile (warpgroup)
-    const int q = warp & 3;              // TMEM lane quadrant
+    // warp w: A tile t = w / 8, column half hc = (w / 4) % 2 of every
+    // accumulator stage, TMEM lane quadrant q = w % 4.  The two column halves
+    // of a lane are merged through shared memory at the end of each item.
+    const int t = warp >> 3;
+    const int hc = (warp >> 2) & 1;
+    const int q = warp & 3;
     const int r = t * 128 + q * 32 + lane;   // A row within the item
-    const int etid = threadIdx.x;        // 0..255
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + hc * 64;
     uint32_t acc_stage = 0, acc_phase = 0;
-    int seg_count = 0;
+    int seg_count = 0, items_done = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      float best = -INFINITY;            // SpecPC: running max over query heads
-      float acc = 0.f;                   // SpecKV: column sum of this key
+
+    auto wait_acc = [&](int which) -> bool {
+      bool w = mbar_wait(&acc_full[acc_stage], acc_phase, abort_v, site(MODE, 2, which));
+      w = __all_sync(0xffffffffu, w);
+      if (w) tc_fence_after();
+      return w;
+    };
+    auto release_acc = [&]() {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc_stage]);
+    };
+    auto next_acc = [&]() {
+      if (++acc_stage == 2) { acc_stage = 0; acc_phase ^= 1; }
+    };
+    auto wait_uniform = [&](uint64_t* bar, uint32_t parity, int which) -> bool {
+      bool w = mbar_wait(bar, parity, abort_v, site(MODE, 3, which));
+      return __all_sync(0xffffffffu, w);
+    };
+    auto arrive_warp = [&](uint64_t* bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
+      // the second column half may not touch the merge buffers (or, for
+      // SpecPC, its head sums) until the first half has consumed the last item's
+      if (hc == 1 && items_done > 0 && !(ok = wait_uniform(&mrg_empty, (items_done - 1) & 1, 0))) break;
+      float2 sacc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // SpecKV column sum
+      float acc_masked = 0.f;
+      float m = -INFINITY, l = 0.f;                                                 // pass-1 row state
+      int item_u = 0, item_row0 = 0;
       for (int seg = 0; ok && seg < nseg; ++seg, ++seg_count) {
         int u, tc, a_row0;
         decode(p, MODE, item, seg, u, tc, a_row0);
+        item_u = u;
+        item_row0 = a_row0;
         const bool active = a_tile_active(p, MODE, a_row0, t);
         if (MODE == MODE_LSE) {
           const int row = a_row0 + r;
           const bool row_ok = active && row < p.rows;
-          const int i = row_ok ? row % p.R : 0;
-          const int c = min(p.n_in, p.c0 + i);
-          float m = -INFINITY, l = 0.f;
+          const int c = min(p.n_in, p.c0 + (row_ok ? row % p.R : 0));
           for (int bt = 0; bt < nb; ++bt) {
-            ok = mbar_wait(&acc_full[acc_stage], acc_phase, abort_v, site(MODE, 2, 0));
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
+            if (!(ok = wait_acc(0))) break;
             if (active) {
-              const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc_stage * 2 + t) * 128;
+              const uint32_t taddr = tbase + (acc_stage * 2 + t) * 128;
               uint32_t va[32], vb[32];
               tmem_ld32(taddr, va);
               tmem_ld32(taddr + 32, vb);
               tmem_ld_wait2(va, vb);
-              const int j0 = bt * 128;
-              if (row_ok) {
-                lse_update(va, j0, c, p.c2, m, l);
-                lse_update(vb, j0 + 32, c, p.c2, m, l);
-              }
-              __syncwarp();
-              tmem_ld32(taddr + 64, va);
-              tmem_ld32(taddr + 96, vb);
-              tmem_ld_wait2(va, vb);
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[acc_stage]);
-              if (row_ok) {
-                lse_update(va, j0 + 64, c, p.c2, m, l);
-                lse_update(vb, j0 + 96, c, p.c2, m, l);
-              }
+              release_acc();
+              if (row_ok) lse_update64(va, vb, bt * 128 + hc * 64, c, p.c2, m, l);
             } else {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&acc_empty[acc_stage]);
+              release_acc();
             }
-            if (++acc_stage == 2) { acc_stage = 0; acc_phase ^= 1; }
-          }
-          if (ok && row_ok) {
-            float out = m + lg2_approx(l);
-            if (p.row_weights != nullptr) out += log2_norm - log2f(p.row_weights[i]);
-            p.lse2[static_cast<size_t>(u) * p.rows + row] = out;
+            next_acc();
           }
         } else {
-          // Load this unit's row offsets (lse2, +inf past the last row) into
-          // buffer seg_count & 1.  Every epilogue thread arrives on
-          // off_ready[buf] after writing; the bounded wait replaces a named
-          // barrier so that an aborting warp cannot strand the others.  A
-          // buffer is rewritten two segments later, after every thread has
-          // passed the wait of the segment in between.
-          const int buf = seg_count & 1;
-          float* off = lse_s + buf * kRowsMax;
-          const int rows_pad = nb * 128;
-          const float* src = p.lse2 + static_cast<size_t>(u) * p.rows;
-          for (int n = etid; n < rows_pad; n += kEpiThreads) off[n] = (n < p.rows) ? src[n] : INFINITY;
-          mbar_arrive(&off_ready[buf]);
-          ok = mbar_wait(&off_ready[buf], (seg_count >> 1) & 1, abort_v, site(MODE, 2, 2));
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
+          // this segment's row offsets (-lse2, -inf on padding rows) arrive by bulk copy
+          const int ob = seg_count & 1;
+          if (!(ok = wait_uniform(&off_full[ob], (seg_count >> 1) & 1, 2))) break;
+          const float* off = off_s + ob * kRowsMax;
           const int j = a_row0 + r;              // this thread's key
           const bool masked_key = j >= p.c0;     // some rows cannot see it
+          const int gh = p.rows / p.R;           // query heads of the unit
+          const int head0 = (seg / p.layers_used) * gh;   // SpecPC: first query head of this KV head
           float seg_sum = 0.f;
           int cur_head = -1;
+          float* my_acc = acc_s + hc * kHeadsMax * 256;
           for (int bt = 0; bt < nb; ++bt) {
-            ok = mbar_wait(&acc_full[acc_stage], acc_phase, abort_v, site(MODE, 2, 1));
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            if (active) {
-              const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc_stage * 2 + t) * 128;
-              const int ncols = chunk_cols(p, bt);
-              for (int g = 0; g < ncols; g += 32) {
-                uint32_t v[32];
-                __syncwarp();
-                tmem_ld32(taddr + g, v);
-                tmem_ld_wait(v);
-                const int nb0 = bt * 128 + g;
-                if (MODE == MODE_COLSUM) {
-                  acc += masked_key ? colsum32_masked(v, off, nb0, p.c2, j, p.c0, p.R) : colsum32(v, off, nb0, p.c2);
+            if (!(ok = wait_acc(1))) break;
+            const int width = active ? min(64, chunk_cols(p, bt) - hc * 64) : 0;   // 0, 32 or 64 columns
+            auto process32 = [&](const uint32_t (&v)[32], int nb0) {
+              if (MODE == MODE_COLSUM) {
+                if (masked_key) acc_masked += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
+                else colsum32(v, off + nb0, p.c2, sacc);
+              } else {
+                // SpecPC: rows of one query head are contiguous (R = W rows);
+                // rows >= p.rows are padding and belong to no head
+                const int h0 = nb0 / p.R, h1 = (nb0 + 31) / p.R;
+                if (h0 >= gh) {
+                  // the whole group is padding
+                } else if (h0 == h1) {
+                  if (h0 != cur_head) {
+                    if (cur_head >= 0) my_acc[(head0 + cur_head) * 256 + r] += seg_sum;
+                    cur_head = h0;
+                    seg_sum = 0.f;
+                  }
+                  if (masked_key) {
+                    seg_sum += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
+                  } else {
+                    float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+                    colsum32(v, off + nb0, p.c2, gs);
+                    seg_sum += fold(gs);
+                  }
                 } else {
-                  // SpecPC: rows of one query head are contiguous (R = W rows);
-                  // rows >= p.rows are padding and belong to no head
-                  const int gh = p.rows / p.R;
-                  const int h0 = nb0 / p.R, h1 = (nb0 + 31) / p.R;
-                  if (h0 >= gh) {
-                    // whole group is padding
-                  } else if (h0 == h1) {
-                    if (h0 != cur_head) {
-                      if (cur_head >= 0) acc_s[cur_head * 256 + r] += seg_sum;
-                      cur_head = h0;
+                  // a 32-row group that straddles two query heads
+                  int i = nb0 % p.R;
+                  for (int k = 0; k < 32; ++k) {
+                    const int n = nb0 + k;
+                    if (n >= p.rows) break;
+                    const int hh = n / p.R;
+                    if (hh != cur_head) {
+                      if (cur_head >= 0) my_acc[(head0 + cur_head) * 256 + r] += seg_sum;
+                      cur_head = hh;
                       seg_sum = 0.f;
                     }
-                    seg_sum += masked_key ? colsum32_masked(v, off, nb0, p.c2, j, p.c0, p.R)
-                                          : colsum32(v, off, nb0, p.c2);
-                  } else {
-                    // a 32-row group that straddles two query heads
-                    int i = nb0 % p.R;
-                    for (int k = 0; k < 32; ++k) {
-                      const int n = nb0 + k;
-                      if (n >= p.rows) break;
-                      const int hh = n / p.R;
-                      if (hh != cur_head) {
-                        if (cur_head >= 0) acc_s[cur_head * 256 + r] += seg_sum;
-                        cur_head = hh;
-                        seg_sum = 0.f;
-                      }
-                      if (!masked_key || j < p.c0 + i)
-                        seg_sum += ex2_approx(fmaf(__uint_as_float(v[k]), p.c2, -off[n]));
-                      if (++i == p.R) i = 0;
-                    }
+                    if (!masked_key || j < p.c0 + i)
+                      seg_sum += ex2_approx(fmaf(__uint_as_float(v[k]), p.c2, off[n]));
+                    if (++i == p.R) i = 0;
                   }
                 }
               }
+            };
+            // 32 columns per TMEM wait keeps the live registers within budget
+            const uint32_t taddr = tbase + (acc_stage * 2 + t) * 128;
+            if (width == 0) release_acc();
+            for (int g = 0; g < width; g += 32) {
+              uint32_t v[32];
+              __syncwarp();
+              tmem_ld32(taddr + g, v);
+              tmem_ld_wait(v);
+              if (g + 32 >= width) release_acc();
+              process32(v, bt * 128 + hc * 64 + g);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc_stage]);
-            if (++acc_stage == 2) { acc_stage = 0; acc_phase ^= 1; }
+            next_acc();
           }
-          if (MODE == MODE_COLSUM_PC && ok && active) {
-            if (cur_head >= 0) acc_s[cur_head * 256 + r] += seg_sum;
-            // after the last layer of this KV head: max over its query heads
-            const int lu = seg % p.layers_used;
-            if (lu == p.layers_used - 1) {
-              const int g = p.rows / p.R;
-              for (int hh = 0; hh < g; ++hh) {
-                best = fmaxf(best, acc_s[hh * 256 + r]);
-                acc_s[hh * 256 + r] = 0.f;
-              }
-            }
-          }
+          // this segment's offsets are no longer read
+          arrive_warp(&off_empty[ob]);
+          if (MODE == MODE_COLSUM_PC && ok && active && cur_head >= 0)
+            my_acc[(head0 + cur_head) * 256 + r] += seg_sum;
         }
       }
       if (!ok) break;
-      if (MODE == MODE_COLSUM) {
-        int u, tc, a_row0;
-        decode(p, MODE, item, 0, u, tc, a_row0);
-        const int j = a_row0 + r;
-        if (a_tile_active(p, MODE, a_row0, t)) {
-          if (j < p.n_pre) p.out0[static_cast<size_t>(u) * p.n_pre + j] = acc;
-          else if (j < p.n_cols && p.out1 != nullptr)
-            p.out1[static_cast<size_t>(u) * (p.n_in - p.n_pre) + (j - p.n_pre)] = acc;
+
+      // ---- merge the two column halves and write this item's outputs
+      if (MODE == MODE_LSE) {
+        if (hc == 1) {
+          xm_s[r] = m;
+          xl_s[r] = l;
+          arrive_warp(&mrg_full);
+        } else {
+          if (!(ok = wait_uniform(&mrg_full, items_done & 1, 1))) break;
+          const float m1 = xm_s[r], l1 = xl_s[r];
+          arrive_warp(&mrg_empty);
+          const int row = item_row0 + r;
+          if (a_tile_active(p, MODE, item_row0, t)) {
+            float* dst = p.lse2 + static_cast<size_t>(item_u) * p.lse_stride;
+            if (row < p.rows) {
+              const float M = fmaxf(m, m1);
+              const float L = l * ex2_approx(m - M) + l1 * ex2_approx(m1 - M);
+              float out = M + lg2_approx(L);
+              if (p.row_weights != nullptr) out += log2_norm - log2f(p.row_weights[row % p.R]);
+              dst[row] = p.lse_store ? -out : out;
+            } else if (p.lse_store && row < p.lse_stride) {
+              dst[row] = -INFINITY;
+            }
+          }
         }
-      } else if (MODE == MODE_COLSUM_PC) {
-        const int b = item / p.n_blocks;
-        const int j = (item % p.n_blocks) * 256 + r;
-        if (j < p.n_cols) p.out0[static_cast<size_t>(b) * p.n_in + j] = best;
+      } else if (MODE == MODE_COLSUM) {
+        const float part = fold(sacc) + acc_masked;
+        if (hc == 1) {
+          xm_s[r] = part;
+          arrive_warp(&mrg_full);
+        } else {
+          if (!(ok = wait_uniform(&mrg_full, items_done & 1, 1))) break;
+          const float total = part + xm_s[r];
+          arrive_warp(&mrg_empty);
+          const int j = item_row0 + r;
+          if (a_tile_active(p, MODE, item_row0, t)) {
+            if (j < p.n_pre) p.out0[static_cast<size_t>(item_u) * p.n_pre + j] = total;
+            else if (j < p.n_cols && p.out1 != nullptr)
+              p.out1[static_cast<size_t>(item_u) * (p.n_in - p.n_pre) + (j - p.n_pre)] = total;
+          }
+        }
+      } else {
+        // SpecPC: both halves' per-head sums are complete; max over query heads
+        if (hc == 1) {
+          arrive_warp(&mrg_full);
+        } else {
+          if (!(ok = wait_uniform(&mrg_full, items_done & 1, 1))) break;
+          const int hq = (p.rows / p.R) * p.hkv;
+          float best = -INFINITY;
+          for (int qh = 0; qh < hq; ++qh) {
+            float* a0 = acc_s + qh * 256 + r;
+            float* a1 = acc_s + (kHeadsMax + qh) * 256 + r;
+            best = fmaxf(best, *a0 + *a1);
+            *a0 = 0.f;
+            *a1 = 0.f;
+          }
+          arrive_warp(&mrg_empty);
+          const int b = item / p.n_blocks;
+          const int j = (item % p.n_blocks) * 256 + r;
+          if (j < p.n_cols) p.out0[static_cast<size_t>(b) * p.n_in + j] = best;
+        }
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);

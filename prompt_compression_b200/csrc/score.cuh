@@ -13,7 +13,7 @@ enum ScoreMode : int {
 };
 
 constexpr int kRowsMax = 2048;   // query rows per unit (g * rows-per-head) held in shared memory
-constexpr int kGroupMax = 16;    // SpecPC: query heads per KV head
+constexpr int kHeadsMax = 32;    // SpecPC: query heads per layer
 
 struct ScoreParams {
   // geometry of a unit (one batch element, layer >= l_skip, KV head)
@@ -34,7 +34,9 @@ struct ScoreParams {
   int n_items;       // persistent-loop items
   int n_blocks;      // items per unit (LSE: 256-row blocks) or per batch/unit (256-key blocks)
   // buffers
-  float* lse2;       // [n_units][rows]: LSE writes it, the column passes read it
+  float* lse2;       // LSE writes it, the column passes read it (see lse_store)
+  int lse_stride;    // floats between units in lse2
+  int lse_store;     // 0: lse2[u][row] as is (rows only); 1: -lse2, rows..lse_stride-1 = -inf
   float* out0;       // SpecKV scores [n_units][n_pre] or SpecPC scores [batch][n_in]
   float* out1;       // SpecKV window mass [n_units][n_in - n_pre] (nullable)
   int n_pre;         // prefix keys that are scored
