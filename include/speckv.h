@@ -197,8 +197,8 @@ const char* spk_last_error(void);
 spk_status spk_device_error(int* status, int* site, int clear);
 
 /* Diagnostic: y[i] = 2^t[i] as computed on the FMA pipe by the scoring
- * epilogues (range reduction + fitted degree-5 polynomial, relative error
- * <= 2.2e-7 for t in [-126, 64); arguments below -126 give a value under
+ * epilogues (range reduction + fitted degree-4 polynomial, relative error
+ * <= 2.7e-6 for t in [-126, 64); arguments below -126 give a value under
  * 1.2e-38).  t, y: fp32 device arrays of n elements. */
 spk_status spk_exp2_fma(const float* t, float* y, int n, void* stream);
 

@@ -9,11 +9,13 @@
 //   contributes nothing to the sums it feeds);
 //   r = t + 1.5*2^23 rounds t to the nearest integer j in r's low mantissa
 //   bits; j = r - 1.5*2^23 exactly; f = t - j lies in [-1/2, 1/2];
-//   2^f ~= p(f), p of degree 5 with coefficients from a Remez fit of the
+//   2^f ~= p(f), p of degree 4 with coefficients from a Remez fit of the
 //   relative error on [-1/2, 1/2] (csrc/fit_exp2.py: max relative error
-//   7.5e-8 exact, 2.1e-7 evaluated in fp32 Horner form);
+//   2.6e-6 exact, 2.7e-6 evaluated in fp32 Horner form);
 //   2^t = p(f) * 2^j is formed by adding j to p's exponent field: the low 9
 //   bits of r's bit pattern are j, so (bits(r) << 23) adds j << 23 (mod 2^32).
+// Per pair: 2 clamps, 3 range-reduction and 4 Horner fp32x2 operations,
+// 2 shift-adds: 11 instructions for 2 exponentials.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -22,13 +24,12 @@ namespace spk {
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
-// Remez coefficients c0..c5 of p(f) ~= 2^f (fp32 bit patterns).
-#define SPK_EXP2_C0 __uint_as_float(0x3f800001u)
-#define SPK_EXP2_C1 __uint_as_float(0x3f317214u)
-#define SPK_EXP2_C2 __uint_as_float(0x3e75fc8cu)
-#define SPK_EXP2_C3 __uint_as_float(0x3d635b72u)
-#define SPK_EXP2_C4 __uint_as_float(0x3c1e8629u)
-#define SPK_EXP2_C5 __uint_as_float(0x3aae0473u)
+// Remez coefficients c0..c4 of p(f) ~= 2^f (fp32 bit patterns).
+#define SPK_EXP2_C0 __uint_as_float(0x3f7ffff4u)
+#define SPK_EXP2_C1 __uint_as_float(0x3f31706eu)
+#define SPK_EXP2_C2 __uint_as_float(0x3e76036du)
+#define SPK_EXP2_C3 __uint_as_float(0x3d650a20u)
+#define SPK_EXP2_C4 __uint_as_float(0x3c1ccbebu)
 
 __device__ __forceinline__ float2 exp2_fma_pair(float2 t) {
   t.x = fmaxf(t.x, -126.f);
@@ -37,8 +38,7 @@ __device__ __forceinline__ float2 exp2_fma_pair(float2 t) {
   const float2 r = __fadd2_rn(t, f2(kRound, kRound));
   const float2 j = __fadd2_rn(r, f2(-kRound, -kRound));
   const float2 f = __ffma2_rn(j, f2(-1.f, -1.f), t);
-  float2 p = __ffma2_rn(f2(SPK_EXP2_C5, SPK_EXP2_C5), f, f2(SPK_EXP2_C4, SPK_EXP2_C4));
-  p = __ffma2_rn(p, f, f2(SPK_EXP2_C3, SPK_EXP2_C3));
+  float2 p = __ffma2_rn(f2(SPK_EXP2_C4, SPK_EXP2_C4), f, f2(SPK_EXP2_C3, SPK_EXP2_C3));
   p = __ffma2_rn(p, f, f2(SPK_EXP2_C2, SPK_EXP2_C2));
   p = __ffma2_rn(p, f, f2(SPK_EXP2_C1, SPK_EXP2_C1));
   p = __ffma2_rn(p, f, f2(SPK_EXP2_C0, SPK_EXP2_C0));
@@ -51,17 +51,6 @@ __device__ __forceinline__ float2 exp2_mufu_pair(float2 t) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(a) : "f"(t.x));
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(b) : "f"(t.y));
   return f2(a, b);
-}
-
-// Pair p of a run of pairs goes to the FMA pipe when (p & 7) < kPolyPairsOf8:
-// 3 of every 8 pairs (37.5 %) balances 8 FMA-pipe ops per polynomial
-// exponential against the MUFU's 16 exponentials per clock.
-constexpr int kPolyPairsOf8 = 3;
-
-template <int P>
-__device__ __forceinline__ float2 exp2_pair(float2 t) {
-  if constexpr ((P & 7) < kPolyPairsOf8) return exp2_fma_pair(t);
-  else return exp2_mufu_pair(t);
 }
 
 }  // namespace spk

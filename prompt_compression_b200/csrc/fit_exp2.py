@@ -1,7 +1,7 @@
 """Fit the polynomial used by the FMA-pipe exp2 in the scoring epilogue.
 
 2^x = 2^j * 2^f with j = round(x) and f = x - j in [-1/2, 1/2].  2^f is
-approximated by a degree-5 polynomial p whose coefficients minimise the
+approximated by a degree-4 polynomial p whose coefficients minimise the
 maximum RELATIVE error max |p(f) / 2^f - 1| on [-1/2, 1/2]; they are found
 with the Remez exchange algorithm (equioscillation of the weighted error at
 n + 2 reference points), written here from its textbook statement.
@@ -13,7 +13,7 @@ polynomial compares the kernel's results against ex2.approx and exp2f.
 """
 import numpy as np
 
-DEG = 5
+DEG = 4
 A, B = -0.5, 0.5
 
 

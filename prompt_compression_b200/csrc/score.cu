@@ -24,10 +24,12 @@
 //               and one 64-column half of every accumulator stage (four warps
 //               per SM sub-partition hide the latency of the exp2 chains); the
 //               two halves of a lane are merged in shared memory per item.
-// TMEM holds 2 accumulator stages x 2 A tiles x 128 fp32 columns (512 cols).
-// The epilogues work on 64 columns per TMEM wait with packed fp32x2 math;
-// 3 of every 8 exponential pairs run on the FMA pipe (exp2_poly.cuh), the
-// rest on the MUFU, so that neither unit alone bounds the pass.
+// TMEM (512 columns): the item's two A tiles (copied from shared memory with
+// tcgen05.cp, so the UMMAs read only B from shared memory) and three
+// 128-column fp32 accumulator buffers that the two tiles use in rotation.
+// The epilogues use packed fp32x2 math; 3/8 of the exponentials run on the
+// FMA pipe (exp2_poly.cuh) and the rest on the MUFU, so that neither unit
+// alone bounds the pass.
 // No atomics: every output element is reduced by exactly one thread in a
 // fixed order, so results are bitwise reproducible.
 #include "common.cuh"
@@ -48,6 +50,11 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 18 * 32;
+
+// Exponential pairs p with (p & 7) < kPolyPairsOf8 run on the FMA pipe
+// (exp2_poly.cuh), the others on the MUFU: 3 of 8 balances the MUFU's 16
+// exponentials per clock against ~7 FMA-pipe operations per polynomial one.
+constexpr int kPolyPairsOf8 = 3;
 
 template <int MODE, int D>
 struct Cfg {
@@ -109,20 +116,9 @@ __device__ __forceinline__ int chunk_cols(const ScoreParams& p, int bt) {
 // ---------------------------------------------------------------------------
 // pass-1 epilogue: online log2-sum-exp2 over 64 keys (jb .. jb+63) of one row
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void lse_update64(const uint32_t (&va)[32], const uint32_t (&vb)[32], int jb, int c,
-                                             float c2, float& m, float& l) {
-  if (jb >= c) return;
-  float x[64];
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    x[k] = __uint_as_float(va[k]);
-    x[32 + k] = __uint_as_float(vb[k]);
-  }
-  if (jb + 64 > c) {
-#pragma unroll
-    for (int k = 0; k < 64; ++k)
-      if (jb + k >= c) x[k] = -INFINITY;
-  }
+// Mask-free core: every one of the 64 logits x is visible (or already -inf).
+template <int POLY_OF_8>
+__device__ __forceinline__ void lse_core64(const float (&x)[64], float c2, float& m, float& l) {
   float a0 = fmaxf(x[0], x[1]), a1 = fmaxf(x[2], x[3]), a2 = fmaxf(x[4], x[5]), a3 = fmaxf(x[6], x[7]);
 #pragma unroll
   for (int k = 8; k < 64; k += 8) {
@@ -138,7 +134,7 @@ __device__ __forceinline__ void lse_update64(const uint32_t (&va)[32], const uin
 #pragma unroll
   for (int p = 0; p < 32; ++p) {
     const float2 t = __ffma2_rn(f2(x[2 * p], x[2 * p + 1]), c2v, nm);
-    const float2 e = ((p & 7) < kPolyPairsOf8) ? exp2_fma_pair(t) : exp2_mufu_pair(t);
+    const float2 e = ((p & 7) < POLY_OF_8) ? exp2_fma_pair(t) : exp2_mufu_pair(t);
     s[p & 3] = __fadd2_rn(s[p & 3], e);
   }
   const float2 s01 = __fadd2_rn(__fadd2_rn(s[0], s[1]), __fadd2_rn(s[2], s[3]));
@@ -147,9 +143,35 @@ __device__ __forceinline__ void lse_update64(const uint32_t (&va)[32], const uin
   m = mn;
 }
 
+// Keys jb .. jb+63 of a row that sees keys [0, c).  Tiles that straddle c
+// take a separate masked copy, so the common path carries no per-key
+// compare/select.
+template <int POLY_OF_8>
+__device__ __forceinline__ void lse_update64(const uint32_t (&va)[32], const uint32_t (&vb)[32], int jb, int c,
+                                             float c2, float& m, float& l) {
+  if (jb >= c) return;
+  float x[64];
+  if (jb + 64 <= c) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      x[k] = __uint_as_float(va[k]);
+      x[32 + k] = __uint_as_float(vb[k]);
+    }
+    lse_core64<POLY_OF_8>(x, c2, m, l);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      x[k] = (jb + k < c) ? __uint_as_float(va[k]) : -INFINITY;
+      x[32 + k] = (jb + 32 + k < c) ? __uint_as_float(vb[k]) : -INFINITY;
+    }
+    lse_core64<POLY_OF_8>(x, c2, m, l);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // pass-2 epilogue: s += 2^(c2 x + off[row]) over 32 rows, off = -lse2
 // ---------------------------------------------------------------------------
+template <int POLY_OF_8>
 __device__ __forceinline__ void colsum32(const uint32_t (&v)[32], const float* off, float c2, float2 (&s)[4]) {
   const float4* o4 = reinterpret_cast<const float4*>(off);
   const float2 c2v = f2(c2, c2);
@@ -160,8 +182,8 @@ __device__ __forceinline__ void colsum32(const uint32_t (&v)[32], const float* o
     const float2 t1 =
         __ffma2_rn(f2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), c2v, f2(o.z, o.w));
     const int p0 = 2 * q, p1 = 2 * q + 1;
-    const float2 e0 = ((p0 & 7) < kPolyPairsOf8) ? exp2_fma_pair(t0) : exp2_mufu_pair(t0);
-    const float2 e1 = ((p1 & 7) < kPolyPairsOf8) ? exp2_fma_pair(t1) : exp2_mufu_pair(t1);
+    const float2 e0 = ((p0 & 7) < POLY_OF_8) ? exp2_fma_pair(t0) : exp2_mufu_pair(t0);
+    const float2 e1 = ((p1 & 7) < POLY_OF_8) ? exp2_fma_pair(t1) : exp2_mufu_pair(t1);
     s[p0 & 3] = __fadd2_rn(s[p0 & 3], e0);
     s[p1 & 3] = __fadd2_rn(s[p1 & 3], e1);
   }
@@ -202,8 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* const off_s = reinterpret_cast<float*>(B_s + C::kSmemB);   // 2 x kRowsMax row offsets
   float* const acc_s = off_s + C::kLseFloats;                         // SpecPC: [2][kHeadsMax][256]
 
-  __shared__ __align__(8) uint64_t a_full[2], a_empty[2], b_full[8], b_empty[8], acc_full[2], acc_empty[2],
-      off_full[2], off_empty[2], mrg_full, mrg_empty, done_bar;
+  __shared__ __align__(8) uint64_t a_full[2], a_empty[2], b_full[8], b_empty[8], acc_full[3], acc_empty[3],
+      off_full[2], off_empty[2], mrg_full, mrg_empty, seg_done, done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
   __shared__ float wsum_s[kThreads / 32];
@@ -215,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kAStages; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], 1); }
     for (int s = 0; s < C::kBStages; ++s) { mbar_init(&b_full[s], 1); mbar_init(&b_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps); }
+    for (int s = 0; s < 3; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps / 2); }
+    mbar_init(&seg_done, 1);
     for (int s = 0; s < 2; ++s) { mbar_init(&off_full[s], 1); mbar_init(&off_empty[s], kEpiWarps); }
     mbar_init(&mrg_full, kEpiWarps / 2);
     mbar_init(&mrg_empty, kEpiWarps / 2);
@@ -315,45 +338,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ UMMA issuer
+    // TMEM columns: accumulator buffers 0..2 at 0, 128, 256; the two A tiles at
+    // 384 + t * D/2 (D/2 32-bit columns hold a 128 x D bf16 tile).  Step k of
+    // tile t accumulates into buffer (2k + t) % 3, its ((2k + t) / 3)-th use.
     if (lane == 0) {
-      uint32_t a_stage = 0, a_phase = 0, b_stage = 0, b_phase = 0, acc_stage = 0, acc_phase = 0;
+      uint32_t a_stage = 0, a_phase = 0, b_stage = 0, b_phase = 0;
+      uint32_t step = 0;           // accumulator steps issued by this CTA
+      uint32_t segs = 0;           // segments started by this CTA
       bool ok = true;
+      const uint32_t a_tmem0 = tmem_base + 384;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        for (int seg = 0; ok && seg < nseg; ++seg) {
+        for (int seg = 0; ok && seg < nseg; ++seg, ++segs) {
           int u, tc, a_row0;
           decode(p, MODE, item, seg, u, tc, a_row0);
           const bool act0 = a_tile_active(p, MODE, a_row0, 0);
           const bool act1 = a_tile_active(p, MODE, a_row0, 1);
           if (!(ok = mbar_wait(&a_full[a_stage], a_phase, abort_v, site(MODE, 1, 0)))) break;
+          // the previous segment's UMMAs must have read the TMEM A tiles
+          if (segs > 0 && !(ok = mbar_wait(&seg_done, (segs - 1) & 1, abort_v, site(MODE, 1, 3)))) break;
           tc_fence_after();
-          const uint64_t a_desc0 = sw128_kmajor_desc(smem_u32(A_s + a_stage * C::kABytes));
-          for (int bt = 0; bt < nb; ++bt) {
+          const uint64_t a_sdesc = sw128_kmajor_desc(smem_u32(A_s + a_stage * C::kABytes));
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!(t == 0 ? act0 : act1)) continue;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t koff = ((t * C::kTileBytes) + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+              tmem_cp_128x256b(a_tmem0 + t * (D / 2) + kk * 8, a_sdesc + koff);
+            }
+          }
+          umma_commit(&a_empty[a_stage]);   // the shared-memory A stage is free once copied
+          if (++a_stage == C::kAStages) { a_stage = 0; a_phase ^= 1; }
+          for (int bt = 0; bt < nb; ++bt, ++step) {
             if (!(ok = mbar_wait(&b_full[b_stage], b_phase, abort_v, site(MODE, 1, 1)))) break;
-            if (!(ok = mbar_wait(&acc_empty[acc_stage], acc_phase ^ 1, abort_v, site(MODE, 1, 2)))) break;
-            tc_fence_after();
             const int n = (MODE == MODE_LSE) ? 128 : chunk_cols(p, bt);
             const uint32_t idesc = idesc_bf16_f32(128, n);
             const uint64_t b_desc0 = sw128_kmajor_desc(smem_u32(B_s + b_stage * C::kTileBytes));
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-              if (!(t == 0 ? act0 : act1)) continue;
-              const uint32_t d_tmem = tmem_base + (acc_stage * 2 + t) * 128;
+              const uint32_t use = 2 * step + t;
+              const uint32_t buf = use % 3;
+              if (!(ok = mbar_wait(&acc_empty[buf], ((use / 3) & 1) ^ 1, abort_v, site(MODE, 1, 2)))) break;
+              tc_fence_after();
+              if (t == 0 ? act0 : act1) {
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                // descriptor start addresses advance in 16-byte units
-                const uint64_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                umma_bf16_ss(d_tmem, a_desc0 + ((t * C::kTileBytes) >> 4) + koff, b_desc0 + koff, idesc,
-                             kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint64_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                  umma_bf16_ts(tmem_base + buf * 128, a_tmem0 + t * (D / 2) + kk * 8, b_desc0 + koff, idesc,
+                               kk > 0 ? 1u : 0u);
+                }
               }
+              umma_commit(&acc_full[buf]);
             }
-            umma_commit(&acc_full[acc_stage]);
+            if (!ok) break;
             umma_commit(&b_empty[b_stage]);
             if (++b_stage == C::kBStages) { b_stage = 0; b_phase ^= 1; }
-            if (++acc_stage == 2) { acc_stage = 0; acc_phase ^= 1; }
           }
           if (!ok) break;
-          umma_commit(&a_empty[a_stage]);
-          if (++a_stage == C::kAStages) { a_stage = 0; a_phase ^= 1; }
+          umma_commit(&seg_done);
         }
       }
       // every UMMA this thread issued has finished before TMEM is freed
@@ -371,12 +413,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int r = t * 128 + q * 32 + lane;   // A row within the item
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + hc * 64;
-    uint32_t acc_stage = 0, acc_phase = 0;
+    uint32_t step = 0;               // accumulator steps consumed (same count as the MMA thread)
     int seg_count = 0, items_done = 0;
     bool ok = true;
+    uint32_t acc_buf = t;            // buffer of this tile at the current step: (2 * step + t) % 3
 
     auto wait_acc = [&](int which) -> bool {
-      bool w = mbar_wait(&acc_full[acc_stage], acc_phase, abort_v, site(MODE, 2, which));
+      const uint32_t use = 2 * step + t;
+      bool w = mbar_wait(&acc_full[acc_buf], (use / 3) & 1, abort_v, site(MODE, 2, which));
       w = __all_sync(0xffffffffu, w);
       if (w) tc_fence_after();
       return w;
@@ -384,10 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto release_acc = [&]() {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc_stage]);
+      if (lane == 0) mbar_arrive(&acc_empty[acc_buf]);
     };
     auto next_acc = [&]() {
-      if (++acc_stage == 2) { acc_stage = 0; acc_phase ^= 1; }
+      ++step;
+      acc_buf = (2 * step + t) % 3;
     };
     auto wait_uniform = [&](uint64_t* bar, uint32_t parity, int which) -> bool {
       bool w = mbar_wait(bar, parity, abort_v, site(MODE, 3, which));
@@ -419,13 +464,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = wait_acc(0))) break;
             if (active) {
-              const uint32_t taddr = tbase + (acc_stage * 2 + t) * 128;
+              const uint32_t taddr = tbase + acc_buf * 128;
               uint32_t va[32], vb[32];
               tmem_ld32(taddr, va);
               tmem_ld32(taddr + 32, vb);
               tmem_ld_wait2(va, vb);
               release_acc();
-              if (row_ok) lse_update64(va, vb, bt * 128 + hc * 64, c, p.c2, m, l);
+              if (row_ok) lse_update64<kPolyPairsOf8>(va, vb, bt * 128 + hc * 64, c, p.c2, m, l);
             } else {
               release_acc();
             }
@@ -445,11 +490,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* my_acc = acc_s + hc * kHeadsMax * 256;
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = wait_acc(1))) break;
-            const int width = active ? min(64, chunk_cols(p, bt) - hc * 64) : 0;   // 0, 32 or 64 columns
+            // this warp's columns of the chunk: 0, 32 or 64 (a chunk narrower than
+            // 64 leaves the second half with none; it must still release the buffer)
+            const int width = active ? max(0, min(64, chunk_cols(p, bt) - hc * 64)) : 0;
             auto process32 = [&](const uint32_t (&v)[32], int nb0) {
               if (MODE == MODE_COLSUM) {
                 if (masked_key) acc_masked += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
-                else colsum32(v, off + nb0, p.c2, sacc);
+                else colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, sacc);
               } else {
                 // SpecPC: rows of one query head are contiguous (R = W rows);
                 // rows >= p.rows are padding and belong to no head
@@ -466,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     seg_sum += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
                   } else {
                     float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-                    colsum32(v, off + nb0, p.c2, gs);
+                    colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, gs);
                     seg_sum += fold(gs);
                   }
                 } else {
@@ -489,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             };
             // 32 columns per TMEM wait keeps the live registers within budget
-            const uint32_t taddr = tbase + (acc_stage * 2 + t) * 128;
+            const uint32_t taddr = tbase + acc_buf * 128;
             if (width == 0) release_acc();
             for (int g = 0; g < width; g += 32) {
               uint32_t v[32];
