@@ -41,8 +41,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--config", default=W.QWEN32B_64K.name,
-                    choices=[c.name for c in W.CONFIGS.values() if isinstance(c, W.SpecKVConfig)])
+    ap.add_argument("--config", default=W.QWEN32B_64K.name, choices=list(W.CONFIGS))
     ap.add_argument("--cmax", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -51,12 +50,21 @@ def parse():
     return ap.parse_args()
 
 
-def config_of(args) -> W.SpecKVConfig:
+def config_of(args):
     import dataclasses
     cfg = W.CONFIGS[args.config]
-    if args.cmax is not None:
+    if args.cmax is not None and isinstance(cfg, W.SpecKVConfig):
         cfg = dataclasses.replace(cfg, c_max=args.cmax)
     return cfg
+
+
+def specpc_flops(cfg: W.SpecPCConfig) -> float:
+    """One Q.K^T product over the causally visible keys of every SpecPC row
+    (query position n_in + n_lookahead - 1 - W + i), all query heads and
+    layers >= l_skip: 2 * d * sum_i c_i per (batch, layer, query head)."""
+    c0 = cfg.n_in + cfg.n_lookahead - cfg.n_rows
+    vis = sum(min(cfg.n_in, c0 + i) for i in range(cfg.n_rows))
+    return 2.0 * cfg.head_dim * vis * cfg.batch * cfg.layers_used * cfg.hq
 
 
 def algorithmic_flops(cfg: W.SpecKVConfig) -> float:
@@ -222,12 +230,42 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- multi-rank plumbing
+def rank_seed(seed: int, rank: int) -> int:
+    """Every rank scores its own batch of units (weak scaling): own seed."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar (device time) over all ranks."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, units_tokens: int, steps: int, ms_total_max: float) -> float:
+    """KV-head-tokens per second over all ranks: every rank processed
+    units_tokens per step; the job took the slowest rank's time."""
+    return world * units_tokens * steps / (ms_total_max * 1e-3)
+
+
 # ----------------------------------------------------------------- GPU arm
 def main():
     args = parse()
     cfg = config_of(args)
     if args.impl == "reference":
+        if not isinstance(cfg, W.SpecKVConfig):
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the CPU reference arm times the SpecKV workloads only"}))
+            return
         run_reference(args, cfg)
+        return
+    if not isinstance(cfg, W.SpecKVConfig):
+        run_other(args, cfg)
         return
 
     import torch
@@ -247,7 +285,7 @@ def main():
     import prompt_compression_b200 as P
     from prompt_compression_b200.pipeline import SpeckvBuffers
 
-    seed = args.seed + 1000 * rank
+    seed = rank_seed(args.seed, rank)
     inp = W.speckv_inputs(cfg, seed=seed, device=dev)
     q, k, v = inp["q"], inp["k"], inp["v"]
     buf = SpeckvBuffers(q, k, v, cfg.n_window, cfg.c_max)
@@ -260,12 +298,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -286,9 +320,9 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_ranks(e0.elapsed_time(e1))
     ms_step = ms_total / args.steps
-    value = world * cfg.kv_head_tokens * args.steps / (ms_total * 1e-3)
+    value = whole_job_value(world, cfg.kv_head_tokens, args.steps, ms_total)
 
     # ---- per-kernel timing: pass 1 alone (row LSE), then the whole score call
     lse2 = torch.empty((cfg.units, cfg.g * cfg.rows), dtype=torch.float32, device=dev)
@@ -344,7 +378,7 @@ def main():
     # ---- e2e through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_over_ranks, barrier)
+        e2e = run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_ranks, barrier)
 
     # ---- CPU baseline (oracle), rank 0 at N = 1 only
     cpu = None
@@ -375,6 +409,86 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_other(args, cfg):
+    """SpecPC (scores + pool + top-K prompt tokens over a draft) and the
+    SpecKV-PC cascade (SpecPC on the draft, gather of the target cache, SpecKV
+    on the gathered cache), one GPU, one JSON line."""
+    import torch
+    from prompt_compression_b200 import build
+    build.build_library()
+    import prompt_compression_b200 as P
+    from prompt_compression_b200.pipeline import SpeckvBuffers
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    cascade = isinstance(cfg, W.CascadeConfig)
+    d = cfg.draft if cascade else cfg
+    dr = W.specpc_inputs(d, seed=args.seed, device=dev)
+    w = torch.from_numpy(W.specpc_row_weights(d.n_rows).astype(np.float32)).to(dev)
+    pc_scores = torch.empty((d.batch, d.n_in), dtype=torch.float32, device=dev)
+    pc_idx = torch.empty((d.batch, min(d.keep, d.n_in)), dtype=torch.int32, device=dev)
+    shape = P.binding.specpc_shape(dr["q"], dr["k"], d.l_skip, d.n_lookahead)
+    ws_pc = torch.empty(max(P.specpc_workspace_size(shape), 256), dtype=torch.uint8, device=dev)
+    ws_tk = torch.empty(max(P.topk_workspace_size(d.batch, d.n_in), 256), dtype=torch.uint8, device=dev)
+    flops = 2 * specpc_flops(d)
+    launches_per_step = 3
+    if cascade:
+        t = cfg.target
+        tfull = W.SpecKVConfig("cascade_target_full", batch=t.batch, layers=t.layers, hq=t.hq, hkv=t.hkv,
+                               head_dim=t.head_dim, n_in=cfg.n_in_full, n_window=t.n_window,
+                               n_lookahead=t.n_lookahead, c_max=t.c_max, heavy_frac=t.heavy_frac)
+        tg = W.speckv_inputs(tfull, seed=args.seed + 1, device=dev, heavy_pos=dr["heavy"])
+        kg = torch.empty((t.batch, t.layers, t.hkv, d.keep, t.head_dim), dtype=torch.bfloat16, device=dev)
+        vg = torch.empty_like(kg)
+        buf = SpeckvBuffers(tg["q"], kg, vg, t.n_window, t.c_max)
+        tcfg = W.SpecKVConfig("g", batch=t.batch, layers=t.layers, hq=t.hq, hkv=t.hkv, head_dim=t.head_dim,
+                              n_in=d.keep, n_window=t.n_window, n_lookahead=t.n_lookahead, c_max=t.c_max)
+        flops += 2 * algorithmic_flops(tcfg)
+        launches_per_step += 1 + 4
+        tokens = t.batch * t.layers * t.hkv * cfg.n_in_full
+        metric = "target KV-head-tokens compressed/s (SpecPC 128K -> 2048 -> SpecKV 256 + 64)"
+    else:
+        tokens = d.kv_head_tokens
+        metric = "KV-head-tokens scored+selected/s (SpecPC draft)"
+
+    def step():
+        P.specpc_score(dr["q"], dr["k"], w, pc_scores, d.l_skip, d.n_lookahead, ws_pc, stream=stream)
+        P.topk_select(pc_scores, d.keep, 0, pc_idx, d.pool, None, ws_tk, stream=stream)
+        if cascade:
+            P.kv_compact(tg["k"], tg["v"], pc_idx, kg, vg, t.layers * t.hkv, stream=stream)
+            P.speckv_compress(tg["q"], kg, vg, t.n_window, t.c_max, t.pool, buffers=buf, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, site = P.spk_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} at site {site} during warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        time.sleep(0.3)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": metric, "value": tokens / (ms_step * 1e-3), "unit": "KV-head-tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "tensor", "kernel": "whole step (scoring passes dominate)", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None, "peak_source": f"{peaks['source']} bf16 burst"},
+        "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(), "e2e": None,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_over_ranks, barrier):

@@ -234,7 +234,8 @@ def speckv_inputs(cfg: SpecKVConfig, seed: int = 0, device="cpu", with_v: bool =
 
     Returns dict(q=[B,L,Hq,R,d], k=[B,L,Hkv,n_in,d], v=..., heavy=positions).
     Heavy positions are drawn in [1, n_pre) (the scored prefix), per batch
-    element; u_h is drawn per (batch, layer, KV head).
+    element, unless heavy_pos gives them (one array per batch element); u_h
+    is drawn per (batch, layer, KV head).
     """
     torch = _torch()
     B, L, Hq, Hkv, d = cfg.batch, cfg.layers, cfg.hq, cfg.hkv, cfg.head_dim
@@ -245,7 +246,7 @@ def speckv_inputs(cfg: SpecKVConfig, seed: int = 0, device="cpu", with_v: bool =
     v = torch.empty_like(k) if with_v else None
     heavy = []
     for b in range(B):
-        hp = heavy_pos if heavy_pos is not None else heavy_positions(
+        hp = heavy_pos[b] if heavy_pos is not None else heavy_positions(
             max(cfg.n_pre, 2), cfg.heavy_frac, cfg.heavy_spans, cfg.span_len, seed * 1000 + b)
         heavy.append(np.asarray(hp, dtype=np.int64))
     inv = 1.0 / math.sqrt(d)
