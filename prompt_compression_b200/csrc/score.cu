@@ -52,9 +52,10 @@ constexpr int kMmaWarp = 17;
 constexpr int kThreads = 18 * 32;
 
 // Exponential pairs p with (p & 7) < kPolyPairsOf8 run on the FMA pipe
-// (exp2_poly.cuh), the others on the MUFU: 3 of 8 balances the MUFU's 16
-// exponentials per clock against ~7 FMA-pipe operations per polynomial one.
-constexpr int kPolyPairsOf8 = 3;
+// (exp2_poly.cuh), the others on the MUFU: 2 of 8 (25 %) measured best
+// against the MUFU's 16 exponentials per clock and the ~12 issue slots of a
+// polynomial pair.
+constexpr int kPolyPairsOf8 = 2;
 
 template <int MODE, int D>
 struct Cfg {
@@ -68,6 +69,12 @@ struct Cfg {
   static constexpr int kLseFloats = (MODE == MODE_LSE) ? 0 : 2 * kRowsMax;
   static constexpr int kAccFloats = (MODE == MODE_COLSUM_PC) ? 2 * kHeadsMax * 256 : 0;
   static constexpr int kSmemBytes = 1024 + kSmemA + kSmemB + 4 * (kLseFloats + kAccFloats);
+  // Pass 1 items are long (all keys of a unit): its A tiles live in TMEM and
+  // the UMMAs read only B from shared memory; three accumulator buffers fill
+  // the rest of TMEM.  The column passes change A every few steps: A stays in
+  // (double-buffered) shared memory and four accumulator buffers rotate.
+  static constexpr bool kATmem = (MODE == MODE_LSE);
+  static constexpr uint32_t kNumAcc = kATmem ? 3 : 4;
 };
 
 // Error sites: mode * 100 + role * 10 + barrier.
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* const off_s = reinterpret_cast<float*>(B_s + C::kSmemB);   // 2 x kRowsMax row offsets
   float* const acc_s = off_s + C::kLseFloats;                         // SpecPC: [2][kHeadsMax][256]
 
-  __shared__ __align__(8) uint64_t a_full[2], a_empty[2], b_full[8], b_empty[8], acc_full[3], acc_empty[3],
+  __shared__ __align__(8) uint64_t a_full[2], a_empty[2], b_full[8], b_empty[8], acc_full[4], acc_empty[4],
       off_full[2], off_empty[2], mrg_full, mrg_empty, seg_done, done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
@@ -237,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kAStages; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], 1); }
     for (int s = 0; s < C::kBStages; ++s) { mbar_init(&b_full[s], 1); mbar_init(&b_empty[s], 1); }
-    for (int s = 0; s < 3; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps / 2); }
+    for (int s = 0; s < (int)C::kNumAcc; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps / 2); }
     mbar_init(&seg_done, 1);
     for (int s = 0; s < 2; ++s) { mbar_init(&off_full[s], 1); mbar_init(&off_empty[s], kEpiWarps); }
     mbar_init(&mrg_full, kEpiWarps / 2);
@@ -338,9 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ UMMA issuer
-    // TMEM columns: accumulator buffers 0..2 at 0, 128, 256; the two A tiles at
-    // 384 + t * D/2 (D/2 32-bit columns hold a 128 x D bf16 tile).  Step k of
-    // tile t accumulates into buffer (2k + t) % 3, its ((2k + t) / 3)-th use.
+    // TMEM columns: accumulator buffers at 128 * b; with A in TMEM (pass 1)
+    // the two A tiles sit at 384 + t * D/2 (D/2 32-bit columns hold a 128 x D
+    // bf16 tile).  Step k of tile t accumulates into buffer (2k + t) % kNumAcc,
+    // its ((2k + t) / kNumAcc)-th use.
     if (lane == 0) {
       uint32_t a_stage = 0, a_phase = 0, b_stage = 0, b_phase = 0;
       uint32_t step = 0;           // accumulator steps issued by this CTA
@@ -354,21 +362,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool act0 = a_tile_active(p, MODE, a_row0, 0);
           const bool act1 = a_tile_active(p, MODE, a_row0, 1);
           if (!(ok = mbar_wait(&a_full[a_stage], a_phase, abort_v, site(MODE, 1, 0)))) break;
-          // the previous segment's UMMAs must have read the TMEM A tiles
-          if (segs > 0 && !(ok = mbar_wait(&seg_done, (segs - 1) & 1, abort_v, site(MODE, 1, 3)))) break;
-          tc_fence_after();
           const uint64_t a_sdesc = sw128_kmajor_desc(smem_u32(A_s + a_stage * C::kABytes));
+          if (C::kATmem) {
+            // the previous segment's UMMAs must have read the TMEM A tiles
+            if (segs > 0 && !(ok = mbar_wait(&seg_done, (segs - 1) & 1, abort_v, site(MODE, 1, 3)))) break;
+            tc_fence_after();
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!(t == 0 ? act0 : act1)) continue;
+            for (int t = 0; t < 2; ++t) {
+              if (!(t == 0 ? act0 : act1)) continue;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t koff = ((t * C::kTileBytes) + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-              tmem_cp_128x256b(a_tmem0 + t * (D / 2) + kk * 8, a_sdesc + koff);
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t koff = ((t * C::kTileBytes) + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                tmem_cp_128x256b(a_tmem0 + t * (D / 2) + kk * 8, a_sdesc + koff);
+              }
             }
+            umma_commit(&a_empty[a_stage]);   // the shared-memory A stage is free once copied
+          } else {
+            tc_fence_after();
           }
-          umma_commit(&a_empty[a_stage]);   // the shared-memory A stage is free once copied
-          if (++a_stage == C::kAStages) { a_stage = 0; a_phase ^= 1; }
           for (int bt = 0; bt < nb; ++bt, ++step) {
             if (!(ok = mbar_wait(&b_full[b_stage], b_phase, abort_v, site(MODE, 1, 1)))) break;
             const int n = (MODE == MODE_LSE) ? 128 : chunk_cols(p, bt);
@@ -377,15 +388,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
               const uint32_t use = 2 * step + t;
-              const uint32_t buf = use % 3;
-              if (!(ok = mbar_wait(&acc_empty[buf], ((use / 3) & 1) ^ 1, abort_v, site(MODE, 1, 2)))) break;
+              const uint32_t buf = use % C::kNumAcc;
+              if (!(ok = mbar_wait(&acc_empty[buf], ((use / C::kNumAcc) & 1) ^ 1, abort_v, site(MODE, 1, 2))))
+                break;
               tc_fence_after();
               if (t == 0 ? act0 : act1) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                   const uint64_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                  umma_bf16_ts(tmem_base + buf * 128, a_tmem0 + t * (D / 2) + kk * 8, b_desc0 + koff, idesc,
-                               kk > 0 ? 1u : 0u);
+                  if (C::kATmem)
+                    umma_bf16_ts(tmem_base + buf * 128, a_tmem0 + t * (D / 2) + kk * 8, b_desc0 + koff, idesc,
+                                 kk > 0 ? 1u : 0u);
+                  else
+                    umma_bf16_ss(tmem_base + buf * 128, a_sdesc + ((t * C::kTileBytes) >> 4) + koff, b_desc0 + koff,
+                                 idesc, kk > 0 ? 1u : 0u);
                 }
               }
               umma_commit(&acc_full[buf]);
@@ -395,7 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++b_stage == C::kBStages) { b_stage = 0; b_phase ^= 1; }
           }
           if (!ok) break;
-          umma_commit(&seg_done);
+          if (C::kATmem) {
+            umma_commit(&seg_done);
+          } else {
+            umma_commit(&a_empty[a_stage]);   // this segment's UMMAs have read the A stage
+          }
+          if (++a_stage == C::kAStages) { a_stage = 0; a_phase ^= 1; }
         }
       }
       // every UMMA this thread issued has finished before TMEM is freed
@@ -412,15 +433,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hc = (warp >> 2) & 1;
     const int q = warp & 3;
     const int r = t * 128 + q * 32 + lane;   // A row within the item
-    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + hc * 64;
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t step = 0;               // accumulator steps consumed (same count as the MMA thread)
     int seg_count = 0, items_done = 0;
     bool ok = true;
-    uint32_t acc_buf = t;            // buffer of this tile at the current step: (2 * step + t) % 3
+    uint32_t acc_buf = t;            // buffer of this tile at the current step: (2 * step + t) % kNumAcc
 
     auto wait_acc = [&](int which) -> bool {
       const uint32_t use = 2 * step + t;
-      bool w = mbar_wait(&acc_full[acc_buf], (use / 3) & 1, abort_v, site(MODE, 2, which));
+      bool w = mbar_wait(&acc_full[acc_buf], (use / C::kNumAcc) & 1, abort_v, site(MODE, 2, which));
       w = __all_sync(0xffffffffu, w);
       if (w) tc_fence_after();
       return w;
@@ -432,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto next_acc = [&]() {
       ++step;
-      acc_buf = (2 * step + t) % 3;
+      acc_buf = (2 * step + t) % C::kNumAcc;
     };
     auto wait_uniform = [&](uint64_t* bar, uint32_t parity, int which) -> bool {
       bool w = mbar_wait(bar, parity, abort_v, site(MODE, 3, which));
@@ -464,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = wait_acc(0))) break;
             if (active) {
-              const uint32_t taddr = tbase + acc_buf * 128;
+              const uint32_t taddr = tbase + acc_buf * 128 + hc * 64;
               uint32_t va[32], vb[32];
               tmem_ld32(taddr, va);
               tmem_ld32(taddr + 32, vb);
@@ -490,9 +511,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* my_acc = acc_s + hc * kHeadsMax * 256;
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = wait_acc(1))) break;
-            // this warp's columns of the chunk: 0, 32 or 64 (a chunk narrower than
-            // 64 leaves the second half with none; it must still release the buffer)
-            const int width = active ? max(0, min(64, chunk_cols(p, bt) - hc * 64)) : 0;
+            // this warp's columns of the chunk: the first half takes ncols/2
+            // rounded up to 32, the second the rest (possibly none, and then it
+            // only releases the buffer)
+            const int ncols = chunk_cols(p, bt);
+            const int half = ((ncols >> 1) + 31) & ~31;
+            const int col0 = hc == 0 ? 0 : half;
+            const int width = active ? (hc == 0 ? half : ncols - half) : 0;
             auto process32 = [&](const uint32_t (&v)[32], int nb0) {
               if (MODE == MODE_COLSUM) {
                 if (masked_key) acc_masked += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
@@ -536,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             };
             // 32 columns per TMEM wait keeps the live registers within budget
-            const uint32_t taddr = tbase + acc_buf * 128;
+            const uint32_t taddr = tbase + acc_buf * 128 + col0;
             if (width == 0) release_acc();
             for (int g = 0; g < width; g += 32) {
               uint32_t v[32];
@@ -544,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_ld32(taddr + g, v);
               tmem_ld_wait(v);
               if (g + 32 >= width) release_acc();
-              process32(v, bt * 128 + hc * 64 + g);
+              process32(v, bt * 128 + col0 + g);
             }
             next_acc();
           }
