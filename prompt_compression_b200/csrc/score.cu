@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* const acc_s = off_s + C::kLseFloats;                         // SpecPC: [2][kHeadsMax][256]
 
   __shared__ __align__(8) uint64_t a_full[2], a_empty[2], b_full[8], b_empty[8], acc_full[4], acc_empty[4],
-      off_full[2], off_empty[2], mrg_full, mrg_empty, seg_done, done_bar;
+      off_full[2], off_empty[2], mrg_full[2], mrg_empty[2], seg_done, done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
   __shared__ float wsum_s[kThreads / 32];
@@ -247,8 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < (int)C::kNumAcc; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps / 2); }
     mbar_init(&seg_done, 1);
     for (int s = 0; s < 2; ++s) { mbar_init(&off_full[s], 1); mbar_init(&off_empty[s], kEpiWarps); }
-    mbar_init(&mrg_full, kEpiWarps / 2);
-    mbar_init(&mrg_empty, kEpiWarps / 2);
+    for (int s = 0; s < 2; ++s) { mbar_init(&mrg_full[s], kEpiWarps / 2); mbar_init(&mrg_empty[s], kEpiWarps / 2); }
     mbar_init(&done_bar, 1);
     abort_flag = 0;
     fence_mbar_init();
@@ -463,11 +462,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar);
     };
+    // SpecKV column sums, first half: the item whose second-half partial is
+    // still to be added, and the step that adds it and stores the total
+    float pend_part = 0.f;
+    int pend_u = 0, pend_row0 = 0;
+    auto colsum_flush = [&](int n) -> bool {
+      const int slot = n & 1;
+      if (!wait_uniform(&mrg_full[slot], (n >> 1) & 1, 1)) return false;
+      const float total = pend_part + (slot ? xl_s : xm_s)[r];
+      arrive_warp(&mrg_empty[slot]);
+      const int j = pend_row0 + r;
+      if (a_tile_active(p, MODE, pend_row0, t)) {
+        if (j < p.n_pre) p.out0[static_cast<size_t>(pend_u) * p.n_pre + j] = total;
+        else if (j < p.n_cols && p.out1 != nullptr)
+          p.out1[static_cast<size_t>(pend_u) * (p.n_in - p.n_pre) + (j - p.n_pre)] = total;
+      }
+      return true;
+    };
 
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
       // the second column half may not touch the merge buffers (or, for
       // SpecPC, its head sums) until the first half has consumed the last item's
-      if (hc == 1 && items_done > 0 && !(ok = wait_uniform(&mrg_empty, (items_done - 1) & 1, 0))) break;
+      if (MODE != MODE_COLSUM && hc == 1 && items_done > 0 &&
+          !(ok = wait_uniform(&mrg_empty[0], (items_done - 1) & 1, 0)))
+        break;
       float2 sacc[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};   // SpecKV column sum
       float acc_masked = 0.f;
       float m = -INFINITY, l = 0.f;                                                 // pass-1 row state
@@ -586,11 +604,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (hc == 1) {
           xm_s[r] = m;
           xl_s[r] = l;
-          arrive_warp(&mrg_full);
+          arrive_warp(&mrg_full[0]);
         } else {
-          if (!(ok = wait_uniform(&mrg_full, items_done & 1, 1))) break;
+          if (!(ok = wait_uniform(&mrg_full[0], items_done & 1, 1))) break;
           const float m1 = xm_s[r], l1 = xl_s[r];
-          arrive_warp(&mrg_empty);
+          arrive_warp(&mrg_empty[0]);
           const int row = item_row0 + r;
           if (a_tile_active(p, MODE, item_row0, t)) {
             float* dst = p.lse2 + static_cast<size_t>(item_u) * p.lse_stride;
@@ -606,27 +624,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if (MODE == MODE_COLSUM) {
+        // The halves hand over through two slots, and the first half adds
+        // item n's partials at the end of item n + 1: by then the second half
+        // has long finished item n, so neither half waits for the other.
         const float part = fold(sacc) + acc_masked;
+        const int slot = items_done & 1;
         if (hc == 1) {
-          xm_s[r] = part;
-          arrive_warp(&mrg_full);
+          if (items_done >= 2 && !(ok = wait_uniform(&mrg_empty[slot], ((items_done - 2) >> 1) & 1, 0))) break;
+          (slot ? xl_s : xm_s)[r] = part;
+          arrive_warp(&mrg_full[slot]);
         } else {
-          if (!(ok = wait_uniform(&mrg_full, items_done & 1, 1))) break;
-          const float total = part + xm_s[r];
-          arrive_warp(&mrg_empty);
-          const int j = item_row0 + r;
-          if (a_tile_active(p, MODE, item_row0, t)) {
-            if (j < p.n_pre) p.out0[static_cast<size_t>(item_u) * p.n_pre + j] = total;
-            else if (j < p.n_cols && p.out1 != nullptr)
-              p.out1[static_cast<size_t>(item_u) * (p.n_in - p.n_pre) + (j - p.n_pre)] = total;
-          }
+          if (items_done >= 1 && !(ok = colsum_flush(items_done - 1))) break;
+          pend_part = part;
+          pend_u = item_u;
+          pend_row0 = item_row0;
         }
       } else {
         // SpecPC: both halves' per-head sums are complete; max over query heads
         if (hc == 1) {
-          arrive_warp(&mrg_full);
+          arrive_warp(&mrg_full[0]);
         } else {
-          if (!(ok = wait_uniform(&mrg_full, items_done & 1, 1))) break;
+          if (!(ok = wait_uniform(&mrg_full[0], items_done & 1, 1))) break;
           const int hq = (p.rows / p.R) * p.hkv;
           float best = -INFINITY;
           for (int qh = 0; qh < hq; ++qh) {
@@ -636,13 +654,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             *a0 = 0.f;
             *a1 = 0.f;
           }
-          arrive_warp(&mrg_empty);
+          arrive_warp(&mrg_empty[0]);
           const int b = item / p.n_blocks;
           const int j = (item % p.n_blocks) * 256 + r;
           if (j < p.n_cols) p.out0[static_cast<size_t>(b) * p.n_in + j] = best;
         }
       }
     }
+    // the last item's total
+    if (MODE == MODE_COLSUM && ok && hc == 0 && items_done > 0) colsum_flush(items_done - 1);
   }
 
   tc_fence_before();
