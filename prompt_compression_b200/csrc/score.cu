@@ -178,16 +178,26 @@ __device__ __forceinline__ void lse_update64(const uint32_t (&va)[32], const uin
 // ---------------------------------------------------------------------------
 // pass-2 epilogue: s += 2^(c2 x + off[row]) over 32 rows, off = -lse2
 // ---------------------------------------------------------------------------
-template <int POLY_OF_8>
-__device__ __forceinline__ void colsum32(const uint32_t (&v)[32], const float* off, float c2, float2 (&s)[4]) {
+// CUT: the first `cut` (0..32) of the 32 rows cannot see this thread's key;
+// their exponent becomes -inf (MUFU: exactly 0; FMA pipe: 2^-126, far below
+// the rounding of any sum it joins).  With cut = 0 the arithmetic, and so the
+// result, is bit for bit that of the unmasked form.
+template <int POLY_OF_8, bool CUT = false>
+__device__ __forceinline__ void colsum32(const uint32_t (&v)[32], const float* off, float c2, float2 (&s)[4],
+                                         int cut = 0) {
   const float4* o4 = reinterpret_cast<const float4*>(off);
   const float2 c2v = f2(c2, c2);
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const float4 o = o4[q];
-    const float2 t0 = __ffma2_rn(f2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), c2v, f2(o.x, o.y));
-    const float2 t1 =
-        __ffma2_rn(f2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), c2v, f2(o.z, o.w));
+    float2 t0 = __ffma2_rn(f2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), c2v, f2(o.x, o.y));
+    float2 t1 = __ffma2_rn(f2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), c2v, f2(o.z, o.w));
+    if (CUT) {
+      if (4 * q + 0 < cut) t0.x = -INFINITY;
+      if (4 * q + 1 < cut) t0.y = -INFINITY;
+      if (4 * q + 2 < cut) t1.x = -INFINITY;
+      if (4 * q + 3 < cut) t1.y = -INFINITY;
+    }
     const int p0 = 2 * q, p1 = 2 * q + 1;
     const float2 e0 = ((p0 & 7) < POLY_OF_8) ? exp2_fma_pair(t0) : exp2_mufu_pair(t0);
     const float2 e1 = ((p1 & 7) < POLY_OF_8) ? exp2_fma_pair(t1) : exp2_mufu_pair(t1);
@@ -522,6 +532,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float* off = off_s + ob * kRowsMax;
           const int j = a_row0 + r;              // this thread's key
           const bool masked_key = j >= p.c0;     // some rows cannot see it
+          // Rows with head-local index i <= j - c0 cannot see key j.  The
+          // warp's keys are consecutive, so per 32-row group (that stays in
+          // one head) the warp can tell whether no row, every row or a
+          // leading part of the rows is masked for its keys.
+          // (Only m_lane stays live through the loop; the warp-wide facts are
+          // recomputed per group, which costs a vote in the common case.)
+          const int m_lane = masked_key ? j - p.c0 : -1;
+          // 0: no row masked, 1: every row masked, 2: leading rows masked,
+          // 3: the group wraps into the next head (per-row test)
+          auto mask_class = [&](int nb0) -> int {
+            if (!__any_sync(0xffffffffu, m_lane >= 0)) return 0;
+            const int i0 = nb0 % p.R;
+            if (i0 + 32 > p.R) return 3;
+            if (__reduce_max_sync(0xffffffffu, m_lane) < i0) return 0;
+            if (__reduce_min_sync(0xffffffffu, m_lane) >= i0 + 31) return 1;
+            return 2;
+          };
           const int gh = p.rows / p.R;           // query heads of the unit
           const int head0 = (seg / p.layers_used) * gh;   // SpecPC: first query head of this KV head
           float seg_sum = 0.f;
@@ -538,8 +565,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int width = active ? (hc == 0 ? half : ncols - half) : 0;
             auto process32 = [&](const uint32_t (&v)[32], int nb0) {
               if (MODE == MODE_COLSUM) {
-                if (masked_key) acc_masked += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
-                else colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, sacc);
+                const int mc = mask_class(nb0);
+                if (mc == 0) {
+                  colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, sacc);
+                } else if (mc == 2) {
+                  colsum32<kPolyPairsOf8, true>(v, off + nb0, p.c2, sacc, min(32, max(0, m_lane - nb0 % p.R + 1)));
+                } else if (mc == 3) {
+                  if (masked_key) acc_masked += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
+                  else colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, sacc);
+                }
               } else {
                 // SpecPC: rows of one query head are contiguous (R = W rows);
                 // rows >= p.rows are padding and belong to no head
@@ -552,11 +586,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cur_head = h0;
                     seg_sum = 0.f;
                   }
-                  if (masked_key) {
-                    seg_sum += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
-                  } else {
+                  // h0 == h1: the group stays in one head
+                  const int mc = mask_class(nb0);
+                  if (mc == 0) {
                     float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
                     colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, gs);
+                    seg_sum += fold(gs);
+                  } else if (mc == 2) {
+                    float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+                    colsum32<kPolyPairsOf8, true>(v, off + nb0, p.c2, gs, min(32, max(0, m_lane - nb0 % p.R + 1)));
                     seg_sum += fold(gs);
                   }
                 } else {
