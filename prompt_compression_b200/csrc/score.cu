@@ -21,15 +21,18 @@
 //               segment's row offsets (-lse2, one bulk copy), B tiles streamed
 //   warp 17   : TMEM allocator + single-thread UMMA issuer (128 x N x 16 bf16)
 //   warps 0-15: epilogue; warp w owns TMEM lane quadrant w % 4 of A tile w / 8
-//               and one 64-column half of every accumulator stage (four warps
+//               and one column half of every accumulator stage (four warps
 //               per SM sub-partition hide the latency of the exp2 chains); the
 //               two halves of a lane are merged in shared memory per item.
-// TMEM (512 columns): the item's two A tiles (copied from shared memory with
-// tcgen05.cp, so the UMMAs read only B from shared memory) and three
-// 128-column fp32 accumulator buffers that the two tiles use in rotation.
-// The epilogues use packed fp32x2 math; 3/8 of the exponentials run on the
-// FMA pipe (exp2_poly.cuh) and the rest on the MUFU, so that neither unit
-// alone bounds the pass.
+// TMEM (512 columns):
+//   pass 1: the item's two A tiles (copied from shared memory with
+//           tcgen05.cp, so the UMMAs read only B from shared memory) and three
+//           128-column fp32 accumulator buffers that the two tiles rotate
+//           through; its items are long, so refilling A is rare.
+//   pass 2: A changes every few steps, so it is read from (double-buffered)
+//           shared memory and four 128-column accumulator buffers rotate.
+// The epilogues use packed fp32x2 math; a share of the exponentials runs on
+// the FMA pipe (exp2_poly.cuh) and the rest on the MUFU.
 // No atomics: every output element is reduced by exactly one thread in a
 // fixed order, so results are bitwise reproducible.
 #include "common.cuh"
@@ -51,10 +54,12 @@ constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 18 * 32;
 
-// Exponential pairs p with (p & 7) < kPolyPairsOf8 run on the FMA pipe
-// (exp2_poly.cuh), the others on the MUFU: 2 of 8 (25 %) measured best
-// against the MUFU's 16 exponentials per clock and the ~12 issue slots of a
-// polynomial pair.
+// Exponential pairs p with (p & 7) < POLY_OF_8 run on the FMA pipe
+// (exp2_poly.cuh), the others on the MUFU (16 exponentials per clock per SM).
+// The board runs at its power cap during these passes, where FMA-pipe
+// polynomials cost clock; the measured best shares are 1 of 8 for the row
+// pass and 2 of 8 for the column passes.
+constexpr int kPolyRowPass = 1;
 constexpr int kPolyPairsOf8 = 2;
 
 template <int MODE, int D>
@@ -519,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_ld32(taddr + 32, vb);
               tmem_ld_wait2(va, vb);
               release_acc();
-              if (row_ok) lse_update64<kPolyPairsOf8>(va, vb, bt * 128 + hc * 64, c, p.c2, m, l);
+              if (row_ok) lse_update64<kPolyRowPass>(va, vb, bt * 128 + hc * 64, c, p.c2, m, l);
             } else {
               release_acc();
             }
