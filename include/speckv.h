@@ -81,6 +81,9 @@ typedef struct {
   float scale; /* multiplies q.k before the softmax (1.0 if q is pre-scaled) */
 } spk_speckv_shape;
 
+/* Workspace: the row offsets pass 1 hands to pass 2, 32 bytes per query row
+ * with each unit's g * R rows rounded up to 128:
+ * units * ceil(g * R / 128) * 4096 bytes (rounded up to 256); 16-byte aligned. */
 size_t speckv_workspace_size(const spk_speckv_shape* shape);
 
 spk_status speckv_score(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16,
@@ -97,12 +100,13 @@ spk_status speckv_row_lse(const spk_speckv_shape* shape, const void* q_bf16, con
  * has no counterpart: this is a deployment variant.  Serving engines that
  * reserve nearly all of HBM for their own KV-cache pool, and plugin hosts
  * that give plugins no access to the CUDA allocator, can neither cudaMalloc
- * nor spare a workspace; this call keeps pass 1's row-LSE scratch in a fixed
- * 4 MiB array inside the library image instead (no allocation of any kind).
+ * nor spare a workspace; this call keeps pass 1's row offsets in a fixed
+ * 16 MiB array inside the library image instead (no allocation of any kind).
  *   - Same shapes, layouts, outputs and rules as speckv_score.
- *   - Rejects (SPK_ERR_UNSUPPORTED, before any launch) shapes needing more
- *     than 1,048,576 floats of scratch: units * (hq/hkv) * (n_window + n_lookahead).
- *   - Every GPU that loads the library holds the 4 MiB until process exit.
+ *   - Rejects (SPK_ERR_UNSUPPORTED, before any launch) shapes whose workspace
+ *     (speckv_workspace_size) would exceed 16 MiB, i.e. more than 524,288
+ *     query rows with each unit's rows rounded up to 128.
+ *   - Every GPU that loads the library holds the 16 MiB until process exit.
  *   - The first call on a device looks up the array's address on that device
  *     (cudaGetSymbolAddress) and caches it: make it before any stream capture.
  *   - All calls share the array, which keeps the last call's contents (every
@@ -135,6 +139,8 @@ typedef struct {
   float scale;
 } spk_specpc_shape;
 
+/* Workspace: units * ceil((hq/hkv) * W / 128) * 4096 bytes (rounded up to
+ * 256), units = batch * (layers - l_skip) * hkv; 16-byte aligned. */
 size_t specpc_workspace_size(const spk_specpc_shape* shape);
 
 spk_status specpc_score(const spk_specpc_shape* shape, const void* q_bf16, const void* k_bf16,

@@ -147,13 +147,17 @@ extern "C" {
 
 const char* spk_last_error(void) { return g_msg; }
 
-// Row offsets between the passes: [units][rows rounded up to 128] floats.
-static long long rows_padded(long long rows) { return (rows + 127) / 128 * 128; }
+// Row offsets between the passes: one kOffBlockBytes block (32 bytes per row)
+// per 128-row tile of each unit.
+static long long row_tiles(long long rows) { return (rows + 127) / 128; }
+static size_t offset_bytes(long long units, long long rows) {
+  return static_cast<size_t>(units) * static_cast<size_t>(row_tiles(rows)) * kOffBlockBytes;
+}
 
 size_t speckv_workspace_size(const spk_speckv_shape* s) {
   SpeckvGeom g;
   if (check_speckv(s, g) != SPK_OK) return 0;
-  return round_up(static_cast<size_t>(g.units) * rows_padded(g.rows) * sizeof(float), 256);
+  return round_up(offset_bytes(g.units, g.rows), 256);
 }
 
 static spk_status speckv_maps(const spk_speckv_shape* s, const void* q, const void* k, const SpeckvGeom& g,
@@ -176,7 +180,6 @@ spk_status speckv_row_lse(const spk_speckv_shape* s, const void* q, const void* 
                               s->layers, 0);
   p.lse2 = lse2;
   p.lse_stride = static_cast<int>(g.rows);
-  p.lse_store = 0;
   st = run_lse(p, qmap, kmap, s->head_dim, static_cast<cudaStream_t>(stream));
   return st == SPK_OK ? ok() : st;
 }
@@ -198,9 +201,8 @@ spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k,
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
                               s->layers, 0);
-  p.lse2 = static_cast<float*>(ws);
-  p.lse_stride = static_cast<int>(rows_padded(g.rows));
-  p.lse_store = 1;
+  p.off_blocks = static_cast<uint8_t*>(ws);
+  p.off_tiles = static_cast<int>(row_tiles(g.rows));
   if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
   p.n_pre = static_cast<int>(g.n_pre);
   p.n_cols = n_cols;
@@ -242,7 +244,7 @@ static spk_status check_specpc(const spk_specpc_shape* s, SpeckvGeom& g) {
 size_t specpc_workspace_size(const spk_specpc_shape* s) {
   SpeckvGeom g;
   if (check_specpc(s, g) != SPK_OK) return 0;
-  return round_up(static_cast<size_t>(g.units) * rows_padded(g.rows) * sizeof(float), 256);
+  return round_up(offset_bytes(g.units, g.rows), 256);
 }
 
 spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k, const float* w, float* scores,
@@ -265,9 +267,8 @@ spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k,
   const int c0 = s->n_in + s->n_lookahead - s->n_rows;
   ScoreParams p = base_params(s->head_dim, s->n_in, g, c0, s->scale, s->hkv, s->layers - s->l_skip, s->layers,
                               s->l_skip);
-  p.lse2 = static_cast<float*>(ws);
-  p.lse_stride = static_cast<int>(rows_padded(g.rows));
-  p.lse_store = 1;
+  p.off_blocks = static_cast<uint8_t*>(ws);
+  p.off_tiles = static_cast<int>(row_tiles(g.rows));
   p.row_weights = w;
   if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
   p.row_weights = nullptr;
@@ -383,15 +384,17 @@ extern "C" spk_status spk_selftest_wait_timeout(long long limit_ns, void* stream
 // that reserve nearly all of HBM up front for their KV-cache pool and hand
 // memory out only through their own allocator, and plugin hosts that give a
 // plugin no access to the CUDA allocator.  They also cannot always find room
-// for a workspace.  This entry point keeps the row-LSE scratch of pass 1 in a
-// fixed array that lives in the library image itself, so a call allocates
-// nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+// for a workspace.  This entry point keeps the row offsets that pass 1 hands
+// to pass 2 in a fixed array that lives in the library image itself, so a
+// call allocates nothing (no cudaMalloc, no cudaFree, no allocating library
+// routine).
 //
 // Limits and behaviour:
-//   - the scratch holds kStaticLseFloats = 1,048,576 floats (4 MiB); a shape
-//     with units * (hq/hkv) * (n_window + n_lookahead) above that is rejected
-//     with SPK_ERR_UNSUPPORTED before anything is launched;
-//   - every GPU that loads the library keeps these 4 MiB until the process exits;
+//   - the scratch holds kStaticOffBytes = 16 MiB, 32 bytes per query row with
+//     each unit's rows rounded up to 128: 524,288 rows (one batch element of
+//     a 64-layer, 8-KV-head, 960-row model); a larger shape is rejected with
+//     SPK_ERR_UNSUPPORTED before anything is launched;
+//   - every GPU that loads the library keeps these 16 MiB until the process exits;
 //   - the first call on each device looks up the array's device address with
 //     that device current (cudaGetSymbolAddress) and caches it; make that
 //     first call before any stream capture;
@@ -404,26 +407,26 @@ extern "C" spk_status spk_selftest_wait_timeout(long long limit_ns, void* stream
 
 namespace spk {
 namespace {
-constexpr long long kStaticLseFloats = 1LL << 20;
+constexpr long long kStaticOffBytes = 1LL << 24;
 constexpr int kMaxDevices = 64;
-static __device__ __align__(256) float g_static_lse2[kStaticLseFloats];
-float* g_static_lse2_addr[kMaxDevices] = {};
-std::mutex g_static_lse2_mu;
+static __device__ __align__(256) uint8_t g_static_off[kStaticOffBytes];
+uint8_t* g_static_off_addr[kMaxDevices] = {};
+std::mutex g_static_off_mu;
 
-// Device address of g_static_lse2 on the current device (looked up once per device).
-spk_status static_lse2_address(float** out) {
+// Device address of g_static_off on the current device (looked up once per device).
+spk_status static_off_address(uint8_t** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(SPK_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kMaxDevices);
-  std::lock_guard<std::mutex> lock(g_static_lse2_mu);
-  if (g_static_lse2_addr[dev] == nullptr) {
+  std::lock_guard<std::mutex> lock(g_static_off_mu);
+  if (g_static_off_addr[dev] == nullptr) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_lse2);
+    e = cudaGetSymbolAddress(&p, g_static_off);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
-    g_static_lse2_addr[dev] = static_cast<float*>(p);
+    g_static_off_addr[dev] = static_cast<uint8_t*>(p);
   }
-  *out = g_static_lse2_addr[dev];
+  *out = g_static_off_addr[dev];
   return SPK_OK;
 }
 }  // namespace
@@ -435,26 +438,24 @@ extern "C" spk_status speckv_score_static_ws(const spk_speckv_shape* s, const vo
   SpeckvGeom g;
   spk_status st = check_speckv(s, g);
   if (st != SPK_OK) return st;
-  const long long need = g.units * rows_padded(g.rows);
-  if (need > kStaticLseFloats)
+  const long long need = static_cast<long long>(offset_bytes(g.units, g.rows));
+  if (need > kStaticOffBytes)
     return fail(SPK_ERR_UNSUPPORTED,
-                "units * (hq/hkv) * (n_window + n_lookahead), rows rounded up to 128, = %lld exceeds the static "
-                "scratch of %lld floats; "
-                "use speckv_score with a workspace",
-                need, kStaticLseFloats);
+                "units * (hq/hkv) * (n_window + n_lookahead) rows, rounded up to 128 per unit, need %lld bytes of "
+                "row offsets and exceed the static scratch of %lld bytes; use speckv_score with a workspace",
+                need, kStaticOffBytes);
   if (g.n_pre > 0 && scores == nullptr) return fail(SPK_ERR_ARG, "scores must be non-NULL when n_window < n_in");
   const int n_cols = static_cast<int>(window_mass ? s->n_in : g.n_pre);
   if (n_cols == 0) return ok();
   CUtensorMap qmap, kmap;
   if ((st = speckv_maps(s, q, k, g, &qmap, &kmap)) != SPK_OK) return st;
-  float* lse2 = nullptr;
-  if ((st = static_lse2_address(&lse2)) != SPK_OK) return st;
+  uint8_t* off = nullptr;
+  if ((st = static_off_address(&off)) != SPK_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
                               s->layers, 0);
-  p.lse2 = lse2;
-  p.lse_stride = static_cast<int>(rows_padded(g.rows));
-  p.lse_store = 1;
+  p.off_blocks = off;
+  p.off_tiles = static_cast<int>(row_tiles(g.rows));
   if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
   p.n_pre = static_cast<int>(g.n_pre);
   p.n_cols = n_cols;

@@ -35,6 +35,8 @@
 // the FMA pipe (exp2_poly.cuh) and the rest on the MUFU.
 // No atomics: every output element is reduced by exactly one thread in a
 // fixed order, so results are bitwise reproducible.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "exp2_poly.cuh"
 #include "score.cuh"
@@ -70,10 +72,15 @@ struct Cfg {
   static constexpr int kBStages = (MODE == MODE_LSE) ? (D == 128 ? 4 : 8) : (D == 128 ? 2 : 4);
   static constexpr int kABytes = 2 * kTileBytes;
   static constexpr int kSmemA = kAStages * kABytes;
-  static constexpr int kSmemB = kBStages * kTileBytes;
-  static constexpr int kLseFloats = (MODE == MODE_LSE) ? 0 : 2 * kRowsMax;
+  // column passes: each B stage also holds its tile's row-offset block, and a
+  // block of ones (the keys' side of the offset K-step) follows the stages
+  static constexpr int kOffBytes = (MODE == MODE_LSE) ? 0 : kOffBlockBytes;
+  static constexpr int kBStageBytes = kTileBytes + kOffBytes;
+  static constexpr int kSmemB = kBStages * kBStageBytes;
+  static constexpr int kOnesBytes = kOffBytes;
   static constexpr int kAccFloats = (MODE == MODE_COLSUM_PC) ? 2 * kHeadsMax * 256 : 0;
-  static constexpr int kSmemBytes = 1024 + kSmemA + kSmemB + 4 * (kLseFloats + kAccFloats);
+  static constexpr int kSmemBytes = 1024 + kSmemA + kSmemB + kOnesBytes + 4 * kAccFloats;
+  static_assert(kBStageBytes % 1024 == 0, "B stages keep the 1024-byte alignment of the swizzled tiles");
   // Pass 1 items are long (all keys of a unit): its A tiles live in TMEM and
   // the UMMAs read only B from shared memory; three accumulator buffers fill
   // the rest of TMEM.  The column passes change A every few steps: A stays in
@@ -181,34 +188,42 @@ __device__ __forceinline__ void lse_update64(const uint32_t (&va)[32], const uin
 }
 
 // ---------------------------------------------------------------------------
-// pass-2 epilogue: s += 2^(c2 x + off[row]) over 32 rows, off = -lse2
+// pass-2 epilogue: s += 2^(c2 x) over 32 rows, where the accumulator x
+// already holds q.k - lse2[row] / c2 (the offset K-step)
 // ---------------------------------------------------------------------------
 // CUT: the first `cut` (0..32) of the 32 rows cannot see this thread's key;
 // their exponent becomes -inf (MUFU: exactly 0; FMA pipe: 2^-126, far below
 // the rounding of any sum it joins).  With cut = 0 the arithmetic, and so the
 // result, is bit for bit that of the unmasked form.
 template <int POLY_OF_8, bool CUT = false>
-__device__ __forceinline__ void colsum32(const uint32_t (&v)[32], const float* off, float c2, float2 (&s)[4],
-                                         int cut = 0) {
-  const float4* o4 = reinterpret_cast<const float4*>(off);
+__device__ __forceinline__ void colsum32(const uint32_t (&v)[32], float c2, float2 (&s)[4], int cut = 0) {
   const float2 c2v = f2(c2, c2);
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const float4 o = o4[q];
-    float2 t0 = __ffma2_rn(f2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])), c2v, f2(o.x, o.y));
-    float2 t1 = __ffma2_rn(f2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])), c2v, f2(o.z, o.w));
+  for (int p = 0; p < 16; ++p) {
+    float2 t = __fmul2_rn(f2(__uint_as_float(v[2 * p]), __uint_as_float(v[2 * p + 1])), c2v);
     if (CUT) {
-      if (4 * q + 0 < cut) t0.x = -INFINITY;
-      if (4 * q + 1 < cut) t0.y = -INFINITY;
-      if (4 * q + 2 < cut) t1.x = -INFINITY;
-      if (4 * q + 3 < cut) t1.y = -INFINITY;
+      if (2 * p + 0 < cut) t.x = -INFINITY;
+      if (2 * p + 1 < cut) t.y = -INFINITY;
     }
-    const int p0 = 2 * q, p1 = 2 * q + 1;
-    const float2 e0 = ((p0 & 7) < POLY_OF_8) ? exp2_fma_pair(t0) : exp2_mufu_pair(t0);
-    const float2 e1 = ((p1 & 7) < POLY_OF_8) ? exp2_fma_pair(t1) : exp2_mufu_pair(t1);
-    s[p0 & 3] = __fadd2_rn(s[p0 & 3], e0);
-    s[p1 & 3] = __fadd2_rn(s[p1 & 3], e1);
+    const float2 e = ((p & 7) < POLY_OF_8) ? exp2_fma_pair(t) : exp2_mufu_pair(t);
+    s[p & 3] = __fadd2_rn(s[p & 3], e);
   }
+}
+
+// Row r (0..127) of a row-offset block (layout: kOffBlockBytes): v split
+// into three bf16 terms, h1 = bf16(v), h2 = bf16(v - h1), h3 = bf16(v - h1 - h2).
+__device__ __forceinline__ void store_offset_row(uint8_t* block, int r, float v) {
+  const __nv_bfloat16 h1 = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h1);
+  const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(h2);
+  const __nv_bfloat16 h3 = __float2bfloat16_rn(r2);
+  const uint32_t w0 = static_cast<uint32_t>(__bfloat16_as_ushort(h1)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(h2)) << 16);
+  const uint32_t w1 = static_cast<uint32_t>(__bfloat16_as_ushort(h3));
+  uint8_t* row = block + (r >> 3) * 256 + (r & 7) * 16;
+  *reinterpret_cast<uint4*>(row) = make_uint4(w0, w1, 0u, 0u);
+  *reinterpret_cast<uint4*>(row + 128) = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ float fold(const float2 (&s)[4]) {
@@ -218,13 +233,12 @@ __device__ __forceinline__ float fold(const float2 (&s)[4]) {
 
 // For a key j that some rows cannot see: row n (head-local i = n % R) sees
 // key j only if j < c0 + i.  nb is the first row of the 32.
-__device__ __forceinline__ float colsum32_masked(const uint32_t (&v)[32], const float* off, int nb, float c2,
-                                                 int j, int c0, int R) {
+__device__ __forceinline__ float colsum32_masked(const uint32_t (&v)[32], int nb, float c2, int j, int c0, int R) {
   float s = 0.f;
   int i = nb % R;
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
-    if (j < c0 + i) s += ex2_approx(fmaf(__uint_as_float(v[k]), c2, off[k]));
+    if (j < c0 + i) s += ex2_approx(__uint_as_float(v[k]) * c2);
     if (++i == R) i = 0;
   }
   return s;
@@ -243,11 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* const A_s = smem;
   uint8_t* const B_s = smem + C::kSmemA;
-  float* const off_s = reinterpret_cast<float*>(B_s + C::kSmemB);   // 2 x kRowsMax row offsets
-  float* const acc_s = off_s + C::kLseFloats;                         // SpecPC: [2][kHeadsMax][256]
+  uint8_t* const ones_s = B_s + C::kSmemB;                                  // column passes: offset K-step, keys' side
+  float* const acc_s = reinterpret_cast<float*>(ones_s + C::kOnesBytes);   // SpecPC: [2][kHeadsMax][256]
 
   __shared__ __align__(8) uint64_t a_full[2], a_empty[2], b_full[8], b_empty[8], acc_full[4], acc_empty[4],
-      off_full[2], off_empty[2], mrg_full[2], mrg_empty[2], seg_done, done_bar;
+      mrg_full[2], mrg_empty[2], seg_done, done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
   __shared__ float wsum_s[kThreads / 32];
@@ -261,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kBStages; ++s) { mbar_init(&b_full[s], 1); mbar_init(&b_empty[s], 1); }
     for (int s = 0; s < (int)C::kNumAcc; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps / 2); }
     mbar_init(&seg_done, 1);
-    for (int s = 0; s < 2; ++s) { mbar_init(&off_full[s], 1); mbar_init(&off_empty[s], kEpiWarps); }
     for (int s = 0; s < 2; ++s) { mbar_init(&mrg_full[s], kEpiWarps / 2); mbar_init(&mrg_empty[s], kEpiWarps / 2); }
     mbar_init(&done_bar, 1);
     abort_flag = 0;
@@ -277,6 +290,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (MODE == MODE_COLSUM_PC && threadIdx.x < kEpiThreads)
     for (int n = threadIdx.x; n < C::kAccFloats; n += kEpiThreads) acc_s[n] = 0.f;
+  if (MODE != MODE_LSE && threadIdx.x < 256) {
+    // ones block: every key row has K-chunk 0 = (1, 1, 1, 0 x 5), chunk 1 = 0
+    // (no-swizzle K-major layout of kOffBlockBytes); made visible to the
+    // tensor pipe (async proxy) before the barrier below
+    const int r = threadIdx.x >> 1, c = threadIdx.x & 1;
+    const uint32_t one = 0x3F80u;   // bf16 1.0
+    const uint4 val = c == 0 ? make_uint4(one | (one << 16), one, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(ones_s + (r >> 3) * 256 + c * 128 + (r & 7) * 16) = val;
+    fence_proxy_async_smem();
+  }
   // Row-weight normaliser for SpecPC pass 1: log2(sum_i w_i * (L - l_skip)).
   float log2_norm = 0.f;
   if (MODE == MODE_LSE && p.row_weights != nullptr) {
@@ -305,7 +328,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t a_stage = 0, a_phase = 0, b_stage = 0, b_phase = 0;
       int a_last[2] = {-1, -1};
       int b_last[8] = {-1, -1, -1, -1, -1, -1, -1, -1};
-      int o_last[2] = {-1, -1};
       int seg_count = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -323,23 +345,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                           tc);
           a_last[a_stage] = static_cast<int>(a_phase);
           if (++a_stage == C::kAStages) { a_stage = 0; a_phase ^= 1; }
-          if (MODE != MODE_LSE) {
-            // this segment's row offsets: -lse2 of unit u, padded with -inf
-            const int ob = seg_count & 1;
-            const uint32_t oph = (seg_count >> 1) & 1;
-            if (!(ok = mbar_wait(&off_empty[ob], oph ^ 1, abort_v, site(MODE, 0, 2)))) break;
-            const uint32_t bytes = static_cast<uint32_t>(p.lse_stride) * 4u;
-            mbar_arrive_expect_tx(&off_full[ob], bytes);
-            bulk_load(off_s + ob * kRowsMax, p.lse2 + static_cast<size_t>(u) * p.lse_stride, bytes, &off_full[ob]);
-            o_last[ob] = static_cast<int>(oph);
-          }
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = mbar_wait(&b_empty[b_stage], b_phase ^ 1, abort_v, site(MODE, 0, 1)))) break;
-            mbar_arrive_expect_tx(&b_full[b_stage], C::kTileBytes);
-            uint8_t* bdst = B_s + b_stage * C::kTileBytes;
+            mbar_arrive_expect_tx(&b_full[b_stage], C::kBStageBytes);
+            uint8_t* bdst = B_s + b_stage * C::kBStageBytes;
 #pragma unroll
             for (int a = 0; a < C::kAtoms; ++a)
               tma_load_3d(bdst + a * 16384, &bmap, &b_full[b_stage], a * 64, bt * 128, tc);
+            if (MODE != MODE_LSE)   // this tile's row-offset block, written by pass 1
+              bulk_load(bdst + C::kTileBytes,
+                        p.off_blocks + (static_cast<size_t>(u) * p.off_tiles + bt) * kOffBlockBytes,
+                        kOffBlockBytes, &b_full[b_stage]);
             b_last[b_stage] = static_cast<int>(b_phase);
             if (++b_stage == C::kBStages) { b_stage = 0; b_phase ^= 1; }
           }
@@ -353,8 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (a_last[s] >= 0) mbar_wait(&a_full[s], a_last[s], &never, site(MODE, 0, 7), 100000000ull);
         for (int s = 0; s < C::kBStages; ++s)
           if (b_last[s] >= 0) mbar_wait(&b_full[s], b_last[s], &never, site(MODE, 0, 8), 100000000ull);
-        for (int s = 0; s < 2; ++s)
-          if (o_last[s] >= 0) mbar_wait(&off_full[s], o_last[s], &never, site(MODE, 0, 9), 100000000ull);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -398,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = mbar_wait(&b_full[b_stage], b_phase, abort_v, site(MODE, 1, 1)))) break;
             const int n = (MODE == MODE_LSE) ? 128 : chunk_cols(p, bt);
             const uint32_t idesc = idesc_bf16_f32(128, n);
-            const uint64_t b_desc0 = sw128_kmajor_desc(smem_u32(B_s + b_stage * C::kTileBytes));
+            const uint64_t b_desc0 = sw128_kmajor_desc(smem_u32(B_s + b_stage * C::kBStageBytes));
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
               const uint32_t use = 2 * step + t;
@@ -416,6 +430,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                   else
                     umma_bf16_ss(tmem_base + buf * 128, a_sdesc + ((t * C::kTileBytes) >> 4) + koff, b_desc0 + koff,
                                  idesc, kk > 0 ? 1u : 0u);
+                }
+                if (MODE != MODE_LSE) {
+                  // offset K-step: ones (keys) x (h1, h2, h3) (query rows) adds
+                  // -lse2[row] / c2 to every logit of the row
+                  umma_bf16_ss(tmem_base + buf * 128, nosw_kmajor_desc(smem_u32(ones_s), 128, 256),
+                               nosw_kmajor_desc(smem_u32(B_s + b_stage * C::kBStageBytes + C::kTileBytes), 128, 256),
+                               idesc, 1u);
                 }
               }
               umma_commit(&acc_full[buf]);
@@ -531,10 +552,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             next_acc();
           }
         } else {
-          // this segment's row offsets (-lse2, -inf on padding rows) arrive by bulk copy
-          const int ob = seg_count & 1;
-          if (!(ok = wait_uniform(&off_full[ob], (seg_count >> 1) & 1, 2))) break;
-          const float* off = off_s + ob * kRowsMax;
           const int j = a_row0 + r;              // this thread's key
           const bool masked_key = j >= p.c0;     // some rows cannot see it
           // Rows with head-local index i <= j - c0 cannot see key j.  The
@@ -572,12 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (MODE == MODE_COLSUM) {
                 const int mc = mask_class(nb0);
                 if (mc == 0) {
-                  colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, sacc);
+                  colsum32<kPolyPairsOf8>(v, p.c2, sacc);
                 } else if (mc == 2) {
-                  colsum32<kPolyPairsOf8, true>(v, off + nb0, p.c2, sacc, min(32, max(0, m_lane - nb0 % p.R + 1)));
+                  colsum32<kPolyPairsOf8, true>(v, p.c2, sacc, min(32, max(0, m_lane - nb0 % p.R + 1)));
                 } else if (mc == 3) {
-                  if (masked_key) acc_masked += colsum32_masked(v, off + nb0, nb0, p.c2, j, p.c0, p.R);
-                  else colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, sacc);
+                  if (masked_key) acc_masked += colsum32_masked(v, nb0, p.c2, j, p.c0, p.R);
+                  else colsum32<kPolyPairsOf8>(v, p.c2, sacc);
                 }
               } else {
                 // SpecPC: rows of one query head are contiguous (R = W rows);
@@ -595,11 +612,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const int mc = mask_class(nb0);
                   if (mc == 0) {
                     float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-                    colsum32<kPolyPairsOf8>(v, off + nb0, p.c2, gs);
+                    colsum32<kPolyPairsOf8>(v, p.c2, gs);
                     seg_sum += fold(gs);
                   } else if (mc == 2) {
                     float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-                    colsum32<kPolyPairsOf8, true>(v, off + nb0, p.c2, gs, min(32, max(0, m_lane - nb0 % p.R + 1)));
+                    colsum32<kPolyPairsOf8, true>(v, p.c2, gs, min(32, max(0, m_lane - nb0 % p.R + 1)));
                     seg_sum += fold(gs);
                   }
                 } else {
@@ -615,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       seg_sum = 0.f;
                     }
                     if (!masked_key || j < p.c0 + i)
-                      seg_sum += ex2_approx(fmaf(__uint_as_float(v[k]), p.c2, off[n]));
+                      seg_sum += ex2_approx(__uint_as_float(v[k]) * p.c2);
                     if (++i == p.R) i = 0;
                   }
                 }
@@ -634,8 +651,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             next_acc();
           }
-          // this segment's offsets are no longer read
-          arrive_warp(&off_empty[ob]);
           if (MODE == MODE_COLSUM_PC && ok && active && cur_head >= 0)
             my_acc[(head0 + cur_head) * 256 + r] += seg_sum;
         }
@@ -654,15 +669,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           arrive_warp(&mrg_empty[0]);
           const int row = item_row0 + r;
           if (a_tile_active(p, MODE, item_row0, t)) {
-            float* dst = p.lse2 + static_cast<size_t>(item_u) * p.lse_stride;
+            float out = 0.f;
             if (row < p.rows) {
               const float M = fmaxf(m, m1);
               const float L = l * ex2_approx(m - M) + l1 * ex2_approx(m1 - M);
-              float out = M + lg2_approx(L);
+              out = M + lg2_approx(L);
               if (p.row_weights != nullptr) out += log2_norm - log2f(p.row_weights[row % p.R]);
-              dst[row] = p.lse_store ? -out : out;
-            } else if (p.lse_store && row < p.lse_stride) {
-              dst[row] = -INFINITY;
+            }
+            if (p.off_blocks != nullptr) {
+              if (row < p.off_tiles * 128)
+                store_offset_row(p.off_blocks + (static_cast<size_t>(item_u) * p.off_tiles + row / 128) * kOffBlockBytes,
+                                 row & 127, row < p.rows ? -out / p.c2 : -1e30f);
+            } else if (row < p.rows) {
+              p.lse2[static_cast<size_t>(item_u) * p.lse_stride + row] = out;
             }
           }
         }

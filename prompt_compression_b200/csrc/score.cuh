@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 namespace spk {
 
@@ -12,7 +13,18 @@ enum ScoreMode : int {
   MODE_COLSUM_PC = 2,  // pass 2, SpecPC: per key, weighted layer/row mean per query head, max over heads
 };
 
-constexpr int kRowsMax = 2048;   // query rows per unit (g * rows-per-head) held in shared memory
+constexpr int kRowsMax = 2048;   // query rows per unit (g * rows-per-head)
+
+// Row-offset block of one 128-row B tile: the column passes need
+// t = c2 * q.k - lse2[row] for every logit.  Instead of adding lse2 in the
+// epilogue, each query row carries v = -lse2[row] / c2 split into three bf16
+// terms (h1 + h2 + h3 = v to ~2^-24 relative), and one extra UMMA K-step
+// against a keys-side block of ones adds them to the accumulator, which then
+// holds q.k + v and only needs the scale c2.  Layout: K-major, no swizzle,
+// 8-row x 16-byte core matrices: row r's K-chunk c (8 bf16) at
+// (r / 8) * 256 + c * 128 + (r % 8) * 16; chunk 0 = (h1, h2, h3, 0 x 5),
+// chunk 1 = 0.  Rows past the unit's rows get v = -1e30 (their terms vanish).
+constexpr int kOffBlockBytes = 4096;
 constexpr int kHeadsMax = 32;    // SpecPC: query heads per layer
 
 struct ScoreParams {
@@ -34,9 +46,13 @@ struct ScoreParams {
   int n_items;       // persistent-loop items
   int n_blocks;      // items per unit (LSE: 256-row blocks) or per batch/unit (256-key blocks)
   // buffers
-  float* lse2;       // LSE writes it, the column passes read it (see lse_store)
+  float* lse2;       // pass 1 without off_blocks: lse2[u * lse_stride + row] (rows only)
   int lse_stride;    // floats between units in lse2
-  int lse_store;     // 0: lse2[u][row] as is (rows only); 1: -lse2, rows..lse_stride-1 = -inf
+  // Row offsets between the passes, as operand blocks of one extra UMMA
+  // K-step (see kOffBlockBytes): pass 1 writes them (when non-null), the
+  // column passes read them.  off_tiles = 128-row tiles per unit.
+  uint8_t* off_blocks;
+  int off_tiles;
   float* out0;       // SpecKV scores [n_units][n_pre] or SpecPC scores [batch][n_in]
   float* out1;       // SpecKV window mass [n_units][n_in - n_pre] (nullable)
   int n_pre;         // prefix keys that are scored

@@ -39,9 +39,9 @@ def test_every_declared_symbol_is_exported(lib):
 def test_workspace_sizes(lib):
     from prompt_compression_b200 import binding as B
     s = B.SpeckvShape(1, 64, 40, 8, 128, 65536, 64, 128, 1.0)
-    assert B.speckv_workspace_size(s) == 512 * 1024 * 4     # rows padded to 128
+    assert B.speckv_workspace_size(s) == 512 * 1024 * 32    # 32 B per row, rows padded to 128
     s = B.SpecpcShape(1, 24, 4, 14, 2, 64, 32768, 256, 1, 1.0)
-    assert B.specpc_workspace_size(s) == 40 * 1792 * 4
+    assert B.specpc_workspace_size(s) == 40 * 1792 * 32
     assert B.topk_workspace_size(512, 65472) == 512 * 65472 * 4
 
 

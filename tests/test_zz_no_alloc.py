@@ -60,10 +60,10 @@ def test_static_scratch_matches_workspace_entry(shape):
 
 def test_static_scratch_rejects_oversized_shapes():
     lib, B = _lib()
-    # 64 layers x 8 KV heads x 5 x 192 rows = 491,520 floats fits; 4 batch elements do not
+    # 64 layers x 8 KV heads x 1024 padded rows x 32 B = 16 MiB fits; 4 batch elements do not
     ok = B.SpeckvShape(1, 64, 40, 8, 128, 65536, 64, 128, 1.0)
     big = B.SpeckvShape(4, 64, 40, 8, 128, 65536, 64, 128, 1.0)
     rc = lib.speckv_score_static_ws(ctypes.byref(big), 256, 256, 256, None, None)
     assert rc == B.SPK_ERR_UNSUPPORTED
     assert "static scratch" in lib.spk_last_error().decode()
-    assert lib.speckv_workspace_size(ctypes.byref(ok)) // 4 <= 1 << 20
+    assert lib.speckv_workspace_size(ctypes.byref(ok)) <= 1 << 24
