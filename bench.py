@@ -430,7 +430,7 @@ def main():
         "config": {"workload": cfg.name, "units": cfg.units, "layers": cfg.layers, "hq": cfg.hq,
                    "hkv": cfg.hkv, "head_dim": cfg.head_dim, "n_in": cfg.n_in, "n_window": cfg.n_window,
                    "n_lookahead": cfg.n_lookahead, "c_max": cfg.c_max, "pool": cfg.pool,
-                   "l2": "inputs larger than L2 (K, V 8.6 GB each at 64K); no flush",
+                   "l2": f"inputs larger than L2 (K, V {k.numel() * 2 / 1e9:.1f} GB each); no flush",
                    "parallelism": f"units sharded, {world} rank(s), no collective"},
         "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
         "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
