@@ -169,6 +169,14 @@ def tensor_peak(peaks):
     return peaks["bf16_tflops"], f"{peaks['source']} bf16 burst"
 
 
+def exp2_peak_per_s():
+    """Exponentials per second the SMs can produce: the MUFU gives 16 ex2 per
+    clock per SM; the FMA pipe (128 lanes) spends 2 lane-ops per logit on the
+    scale and the sum and 7 per polynomial exponential, so the best split
+    (40 % polynomial) reaches 16 / 0.6 = 26.7 exponentials per clock per SM."""
+    return 148 * (16.0 / 0.6) * 1965e6
+
+
 def kernel_source_digest():
     """sha256 over the kernel sources; DRAM traffic captured with ncu is only
     reported while the kernels it was captured from are unchanged."""
@@ -507,14 +515,25 @@ def run_other(args, cfg):
         torch.cuda.synchronize()
     ms_step = e0.elapsed_time(e1) / args.steps
     achieved = flops / (ms_step * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "whole step (scoring passes dominate)", "achieved": achieved,
+                "peak": tensor_peak(peaks)[0], "unit": "TFLOP/s", "frac": achieved / tensor_peak(peaks)[0],
+                "traffic": None, "peak_source": tensor_peak(peaks)[1]}
+    if not cascade:
+        # head_dim 64 halves the tensor work per logit, so the exponential
+        # stream (one exp2 per visible logit per pass) is the binding ceiling
+        exps = 2 * specpc_flops(d) / (2 * d.head_dim)
+        peak_exp = exp2_peak_per_s() / 1e9
+        ach_exp = exps / (ms_step * 1e-3) / 1e9
+        roofline = {"bound": "alu", "kernel": "whole step (scoring passes dominate)", "achieved": ach_exp,
+                    "peak": peak_exp, "unit": "Gexp2/s", "frac": ach_exp / peak_exp, "traffic": None,
+                    "peak_source": "derived: 148 SMs x 26.7 exp2/clk (MUFU 16/clk + FMA-pipe polynomial) x 1965 MHz",
+                    "tensor_frac": achieved / tensor_peak(peaks)[0]}
     line = {
         "metric": metric, "value": tokens / (ms_step * 1e-3), "unit": "KV-head-tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "l2": "inputs larger than L2; no flush"},
-        "roofline": {"bound": "tensor", "kernel": "whole step (scoring passes dominate)", "achieved": achieved,
-                     "peak": tensor_peak(peaks)[0], "unit": "TFLOP/s", "frac": achieved / tensor_peak(peaks)[0],
-                     "traffic": None, "peak_source": tensor_peak(peaks)[1]},
+        "roofline": roofline,
         "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(), "e2e": None,
         "cpu_baseline": None,
     }
