@@ -130,7 +130,7 @@ spk_status speckv_score_static_ws(const spk_speckv_shape* shape, const void* q_b
  *   row_weights  fp32 [W], device, oldest row first, w_i >= 0, sum > 0
  *   scores       fp32 [batch][n_in]
  *
- * Supported: head_dim == 64; hq % hkv == 0; hq / hkv <= 16; (hq/hkv) * W <= 2048;
+ * Supported: head_dim == 64; hq % hkv == 0; hq <= 32; (hq/hkv) * W <= 2048;
  * 0 <= l_skip < layers; 1 <= W <= n_in + n_lookahead - 1; n_lookahead >= 1.
  * ------------------------------------------------------------------------ */
 typedef struct {

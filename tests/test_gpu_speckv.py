@@ -114,6 +114,8 @@ def test_tiny_workload(P):
     (5, 1, 1, 2, 1, 128, 129, 16, 8, 500),       # C_max >= n_pre keeps everything
     (6, 1, 1, 4, 2, 64, 96, 96, 4, 8),           # window covers the whole input
     (7, 1, 3, 5, 1, 128, 2100, 64, 128, 256),    # Qwen-like group: 960 rows, 7.5 row tiles
+    (8, 1, 1, 16, 1, 128, 1500, 64, 64, 200),    # g * R = 2048 rows: the largest unit
+    (9, 1, 1, 32, 2, 64, 777, 48, 80, 64),       # g * R = 2048 with head_dim 64, ragged keys
 ])
 def test_speckv_shapes(P, case):
     seed, B, L, hq, hkv, d, n_in, nw, nl, c_max = case

@@ -40,6 +40,7 @@ def _case(seed, B, L, hq, hkv, d, n_in, Wr):
     (2, 2, 2, 0, 6, 2, 333, 40, 1, 50),      # W not a multiple of 32: groups straddle query heads
     (3, 1, 4, 3, 7, 1, 1030, 256, 1, 200),   # g = 7 query heads of 256 rows (draft-like)
     (4, 1, 2, 1, 2, 2, 257, 17, 3, 64),      # lookahead > 1: rows past the input see every key
+    (5, 1, 2, 1, 32, 4, 600, 256, 1, 80),    # 32 query heads (the most), g * W = 2048 rows
 ])
 def test_specpc_parity(P, case):
     import torch
