@@ -189,6 +189,17 @@ spk_status kv_compact(const void* k, const void* v, int units, int n_src, int he
                       const int32_t* idx, int n_idx, int units_per_idx, void* k_out, void* v_out,
                       void* stream);
 
+/* Device address of page-locked, device-mapped host memory (a deployment
+ * helper; the paper has no counterpart).  k and v of kv_compact may point
+ * into such memory: the gather then reads only the selected rows over the
+ * host link instead of copying the whole cache to the device first.
+ *   host  a pointer into memory from cudaHostAlloc / cudaHostRegister (any
+ *         offset into the allocation)
+ *   *dev  the address kernels use for it (owned by the caller's allocation)
+ * Returns SPK_ERR_CUDA (and leaves *dev untouched) when the memory is not
+ * page-locked and mapped, or no device is present. */
+spk_status spk_mapped_host_pointer(const void* host, void** dev);
+
 /* ------------------------------------------------------------------------
  * Errors
  * ------------------------------------------------------------------------ */

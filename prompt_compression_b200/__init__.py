@@ -19,7 +19,7 @@ from .binding import (  # noqa: F401
     speckv_workspace_size, speckv_score, speckv_row_lse,
     specpc_workspace_size, specpc_score,
     topk_workspace_size, topk_select, kv_compact,
-    spk_device_error, spk_selftest_wait_timeout, spk_exp2_fma,
+    spk_device_error, spk_selftest_wait_timeout, spk_exp2_fma, mapped_host_pointer,
 )
 from .pipeline import speckv_compress, specpc_select, cascade_compress  # noqa: F401
 
@@ -28,6 +28,6 @@ __all__ = [
     "speckv_workspace_size", "speckv_score", "speckv_row_lse",
     "specpc_workspace_size", "specpc_score",
     "topk_workspace_size", "topk_select", "kv_compact",
-    "spk_device_error", "spk_selftest_wait_timeout", "spk_exp2_fma",
+    "spk_device_error", "spk_selftest_wait_timeout", "spk_exp2_fma", "mapped_host_pointer",
     "speckv_compress", "specpc_select", "cascade_compress",
 ]

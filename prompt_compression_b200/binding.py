@@ -69,6 +69,7 @@ def load_library():
         "spk_device_error": (I, [ctypes.POINTER(I), ctypes.POINTER(I), I]),
         "spk_selftest_wait_timeout": (I, [ctypes.c_longlong, vp]),
         "spk_exp2_fma": (I, [vp, vp, I, vp]),
+        "spk_mapped_host_pointer": (I, [vp, ctypes.POINTER(vp)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -102,6 +103,24 @@ def _dev(t: Optional[torch.Tensor], name: str, dtype=None) -> Optional[int]:
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
+
+
+def mapped_host_pointer(t: torch.Tensor) -> int:
+    """Device address of a page-locked host tensor (spk_mapped_host_pointer)."""
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError("expected a page-locked (pinned) host tensor")
+    dev = ctypes.c_void_p()
+    _check(load_library().spk_mapped_host_pointer(ctypes.c_void_p(t.data_ptr()), ctypes.byref(dev)))
+    return int(dev.value)
+
+
+def _src(t: Optional[torch.Tensor], name: str) -> Optional[int]:
+    """A gather source: a CUDA tensor, or a pinned host tensor read in place."""
+    if t is None or t.is_cuda:
+        return _dev(t, name)
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return mapped_host_pointer(t)
 
 
 def _workspace(ws: Optional[torch.Tensor], nbytes: int, device) -> torch.Tensor:
@@ -190,12 +209,13 @@ def topk_select(scores, k: int, n_tail: int, idx, pool_kernel: int = 7, pooled=N
 
 
 def kv_compact(k, v, idx, k_out, v_out, units_per_idx: int = 1, stream=None):
-    """k, v [units, n_src, d] (any 2-byte or 4-byte dtype); idx [units/units_per_idx, n_idx]."""
+    """k, v [units, n_src, d] (any 2-byte or 4-byte dtype); idx [units/units_per_idx, n_idx].
+    k and v may be CUDA tensors or pinned host tensors (gathered in place)."""
     lib = load_library()
     n_src, d = k.shape[-2], k.shape[-1]
     units = k.numel() // (n_src * d) if n_src * d else 0
     n_idx = idx.shape[-1]
-    _check(lib.kv_compact(_dev(k, "k"), _dev(v, "v"), units, n_src, d, k.element_size(),
+    _check(lib.kv_compact(_src(k, "k"), _src(v, "v"), units, n_src, d, k.element_size(),
                           _dev(idx, "idx", torch.int32), n_idx, units_per_idx, _dev(k_out, "k_out"),
                           _dev(v_out, "v_out"), _stream(stream)))
     return k_out, v_out

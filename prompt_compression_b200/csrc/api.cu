@@ -328,6 +328,18 @@ spk_status kv_compact(const void* k, const void* v, int units, int n_src, int he
 }
 
 // ------------------------------------------------------------------ device errors
+spk_status spk_mapped_host_pointer(const void* host, void** dev) {
+  if (host == nullptr || dev == nullptr) return fail(SPK_ERR_ARG, "host and dev must be non-NULL");
+  void* d = nullptr;
+  cudaError_t e = cudaHostGetDevicePointer(&d, const_cast<void*>(host), 0);
+  if (e != cudaSuccess) {
+    cudaGetLastError();   // not sticky: clear it
+    return cuda_fail(e, "host memory is not page-locked and mapped into the device");
+  }
+  *dev = d;
+  return ok();
+}
+
 spk_status spk_device_error(int* status, int* site, int clear) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");

@@ -91,3 +91,15 @@ def test_topk_and_compact_argument_errors(lib):
     assert lib.kv_compact(16, 16, 5, 10, 64, 2, 16, 3, 2, 16, 16, None) == B.SPK_ERR_ARG
     assert lib.kv_compact(16, None, 4, 10, 64, 2, 16, 3, 1, 16, 16, None) == B.SPK_ERR_ARG
     assert lib.kv_compact(24, 16, 4, 10, 64, 2, 16, 3, 1, 16, 16, None) == B.SPK_ERR_ARG
+
+
+def test_mapped_host_pointer_rejects_unmapped_memory(lib):
+    # ordinary (pageable) host memory is not mapped into any device: the call
+    # reports an error and leaves the output alone (here, or on a GPU machine)
+    import numpy as np
+    buf = np.zeros(64, dtype=np.uint8)
+    out = ctypes.c_void_p(12345)
+    rc = lib.spk_mapped_host_pointer(ctypes.c_void_p(buf.ctypes.data), ctypes.byref(out))
+    assert rc != 0
+    assert out.value == 12345
+    assert lib.spk_mapped_host_pointer(None, ctypes.byref(out)) == 1   # SPK_ERR_ARG

@@ -215,6 +215,31 @@ def test_kv_compact_broadcast_and_errors(P):
     assert P.spk_device_error() == (0, 0)
 
 
+def test_kv_compact_from_pinned_host_memory(P):
+    # K on the device, V left in page-locked host memory: the gather reads
+    # only the selected V rows in place and matches the device-resident copy
+    import torch
+    rng = np.random.default_rng(17)
+    units, n_src, d, n_idx = 4, 500, 128, 64
+    kb = rng.integers(0, 2 ** 16, size=(units, n_src, d), dtype=np.uint16)
+    vb = rng.integers(0, 2 ** 16, size=(units, n_src, d), dtype=np.uint16)
+    idx = np.stack([np.sort(rng.choice(n_src, n_idx, replace=False)) for _ in range(units)]).astype(np.int32)
+    k = to_bf16_tensor(kb)
+    vh = to_bf16_tensor(vb, device="cpu").pin_memory()
+    ko = torch.empty((units, n_idx, d), dtype=torch.bfloat16, device="cuda")
+    vo = torch.empty_like(ko)
+    P.kv_compact(k, vh, torch.from_numpy(idx).cuda(), ko, vo)
+    torch.cuda.synchronize()
+    assert P.spk_device_error() == (0, 0)
+    ko_b, vo_b = bits_of(ko), bits_of(vo)
+    for u in range(units):
+        np.testing.assert_array_equal(ko_b[u], kb[u][idx[u]])
+        np.testing.assert_array_equal(vo_b[u], vb[u][idx[u]])
+    # pageable host memory is refused before anything is launched
+    with pytest.raises(ValueError):
+        P.kv_compact(k, to_bf16_tensor(vb, device="cpu"), torch.from_numpy(idx).cuda(), ko, vo)
+
+
 def test_argument_errors_do_not_launch(P):
     import torch
     q = torch.zeros((1, 1, 4, 8, 96), dtype=torch.bfloat16, device="cuda")
