@@ -18,7 +18,7 @@
  *              the first l_skip layers skipped, mean first, then max.
  * and section "损失函数 / 训练策略": SpecPC smooths with local pooling.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent (the kernels take the same ones):
  *   - the softmax of a query row runs over the input keys it can see
  *     causally (a window row at position p sees keys 0..p; a lookahead row
  *     sees every input key); lookahead keys are not input keys;
