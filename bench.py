@@ -179,16 +179,19 @@ def exp2_peak_per_s():
     return 148 * (16.0 / 0.6) * 1965e6
 
 
+# The files that define the scoring kernels and how they are launched.
+SCORING_SOURCES = ("api.cu", "common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh")
+
+
 def kernel_source_digest():
-    """sha256 over the kernel sources; DRAM traffic captured with ncu is only
-    reported while the kernels it was captured from are unchanged."""
+    """sha256 over the scoring kernels' sources (SCORING_SOURCES); the DRAM
+    traffic captured with ncu is only reported while they are unchanged."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "prompt_compression_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for name in SCORING_SOURCES:
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()
 
 
@@ -309,6 +312,9 @@ def main():
                               "the CPU reference arm times the SpecKV workloads only"}))
             return
         run_reference(args, cfg)
+        return
+    if isinstance(cfg, W.DecodeConfig):
+        run_decode(args, cfg)
         return
     if not isinstance(cfg, W.SpecKVConfig):
         run_other(args, cfg)
@@ -538,6 +544,76 @@ def run_other(args, cfg):
         "roofline": roofline,
         "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(), "e2e": None,
         "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_decode(args, cfg):
+    """One decode step over the compressed cache (C_max + window rows per KV
+    head) on every (layer, query head), one JSON line; the same step over the
+    full cache is timed for contrast.  Four copies of the compressed cache are
+    used in rotation so that consecutive launches read 4 x 84 MB, more than
+    the L2; the full cache (17 GB) is far larger than the L2."""
+    import torch
+    from prompt_compression_b200 import build
+    build.build_library()
+    import prompt_compression_b200 as P
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    gen = torch.Generator(device=dev).manual_seed(args.seed)
+    B_, L, hq, hkv, d = cfg.batch, cfg.layers, cfg.hq, cfg.hkv, cfg.head_dim
+
+    def rnd(*shape):
+        return torch.randn(shape, generator=gen, device=dev).to(torch.bfloat16)
+
+    copies = 4
+    qs = [rnd(B_, L, hq, d) for _ in range(copies)]
+    kcs = [rnd(B_, L, hkv, cfg.n_kv, d) for _ in range(copies)]
+    vcs = [rnd(B_, L, hkv, cfg.n_kv, d) for _ in range(copies)]
+    out = torch.empty((B_, L, hq, d), dtype=torch.float32, device=dev)
+    scale = d ** -0.5
+
+    def timed(fn, n):
+        for i in range(max(3, args.warmup)):
+            fn(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    steps = max(args.steps, 20) * 10
+    with ClockSampler(dev.index) as clk:
+        time.sleep(0.3)
+        ms = timed(lambda i: P.decode_attention(qs[i % copies], kcs[i % copies], vcs[i % copies], out, scale,
+                                                stream), steps)
+    st, site = P.spk_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} at site {site}")
+    del kcs, vcs
+    kf, vf = rnd(B_, L, hkv, cfg.n_kv_full, d), rnd(B_, L, hkv, cfg.n_kv_full, d)
+    ms_full = timed(lambda i: P.decode_attention(qs[0], kf, vf, out, scale, stream), max(args.steps, 5))
+    del kf, vf
+    peaks = load_peaks()
+    nbytes = cfg.units * cfg.n_kv * d * 2 * 2 + B_ * L * hq * d * (2 + 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "decode over the compressed cache: query-head tokens/s", "value": B_ * L * hq / (ms * 1e-3),
+        "unit": "query-head tokens/s", "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup),
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "n_kv": cfg.n_kv, "units": cfg.units, "hq": hq, "head_dim": d,
+                   "l2": "4 cache copies in rotation (4 x 84 MB > L2); no flush"},
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peaks['source']} HBM copy"},
+        "full_cache": {"n_kv": cfg.n_kv_full, "ms_per_step": ms_full,
+                       "gbs": cfg.units * cfg.n_kv_full * d * 4 / (ms_full * 1e-3) / 1e9},
+        "gpu_launches": steps, "clocks": clk.summary(), "e2e": None, "cpu_baseline": None,
     }
     print(json.dumps(line), flush=True)
 

@@ -189,6 +189,25 @@ spk_status kv_compact(const void* k, const void* v, int units, int n_src, int he
                       const int32_t* idx, int n_idx, int units_per_idx, void* k_out, void* v_out,
                       void* stream);
 
+/* ------------------------------------------------------------------------
+ * Decode attention over a compacted cache (section 整体框架: the target model
+ * then runs on the compressed KV cache; section 关键设计, SpecKV: the cache
+ * holds the kept KV pairs).  One new query token per attention head:
+ *
+ *   out[b][l][qh][:] = sum_t softmax_t(scale * q[b][l][qh] . k[b][l][qh/g][t]) * v[b][l][qh/g][t]
+ *   q      bf16 [batch][layers][hq][head_dim]
+ *   k, v   bf16 [batch][layers][hkv][n_kv][head_dim]   (e.g. kv_compact's outputs)
+ *   out    fp32 [batch][layers][hq][head_dim]
+ * The softmax runs over all n_kv rows (the caller appends the new token's own
+ * K/V row when it should attend to itself).  Deterministic.
+ *
+ * Supported: head_dim in {64, 128}; hq % hkv == 0; hq / hkv <= 8; n_kv >= 1;
+ * scale > 0 and finite.
+ * ------------------------------------------------------------------------ */
+spk_status decode_attention(int batch, int layers, int hq, int hkv, int head_dim, int n_kv, float scale,
+                            const void* q_bf16, const void* k_bf16, const void* v_bf16, float* out,
+                            void* stream);
+
 /* Device address of page-locked, device-mapped host memory (a deployment
  * helper; the paper has no counterpart).  k and v of kv_compact may point
  * into such memory: the gather then reads only the selected rows over the

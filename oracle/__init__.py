@@ -52,9 +52,10 @@ def _load():
         lib.oracle_maxpool.argtypes = [_dp, I, I, _dp]
         lib.oracle_topk_with_tail.argtypes = [_dp, I, I, I, _i32p]
         lib.oracle_gather_rows.argtypes = [_u8p, I, I, _i32p, I, _u8p]
+        lib.oracle_decode_row.argtypes = [_u16p, _u16p, _u16p, I, I, D, _dp]
         for f in (lib.oracle_speckv_unit, lib.oracle_speckv_unit_f64, lib.oracle_specpc_batch,
                   lib.oracle_specpc_batch_f64, lib.oracle_maxpool, lib.oracle_topk_with_tail,
-                  lib.oracle_gather_rows):
+                  lib.oracle_gather_rows, lib.oracle_decode_row):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -152,6 +153,28 @@ def gather_rows(src, idx):
     _check(lib.oracle_gather_rows(_ptr(src.view(np.uint8), _u8p), n_src, row_bytes,
                                   _ptr(idx, _i32p), idx.size, _ptr(dst.view(np.uint8), _u8p)))
     return dst
+
+
+def decode_attention(q, k, v, scale: float = 1.0):
+    """Decode attention over a compacted cache, every (batch, layer, query head):
+    q [B][L][Hq][d], k/v [B][L][Hkv][n_kv][d] (bf16 bit patterns) -> out
+    [B][L][Hq][d] in float64; query head qh reads KV head qh // (Hq // Hkv)."""
+    lib = _load()
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    B, L, hq, d = q.shape
+    hkv, n_kv = k.shape[2], k.shape[3]
+    g = hq // hkv
+    out = np.zeros((B, L, hq, d), np.float64)
+    for b in range(B):
+        for l in range(L):
+            for qh in range(hq):
+                row = np.zeros(d, np.float64)
+                _check(lib.oracle_decode_row(_ptr(q[b, l, qh], _u16p), _ptr(k[b, l, qh // g], _u16p),
+                                             _ptr(v[b, l, qh // g], _u16p), n_kv, d, scale, _ptr(row, _dp)))
+                out[b, l, qh] = row
+    return out
 
 
 def speckv_select_unit(q, k, n_window, n_lookahead, c_max, pool=7, scale=1.0):

@@ -253,3 +253,38 @@ int oracle_gather_rows(const uint8_t *src, int n_src, int row_bytes, const int32
     }
     return 0;
 }
+
+/*
+ * Decode attention over a compacted cache ("Draft-based Approximate Inference
+ * for LLMs", paper notes, section 整体框架: the target model runs on the
+ * compressed KV cache; section 关键设计, SpecKV: that cache holds the kept
+ * KV pairs).  One query row of one head against n_kv rows of its KV head:
+ *   z_t = scale * <q, k_t>,  p_t = exp(z_t - max z) / sum exp(z - max z),
+ *   out = sum_t p_t v_t.
+ * q [d], k [n_kv][d], v [n_kv][d] as bf16 bit patterns; out [d] in double.
+ */
+int oracle_decode_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, int n_kv, int d, double scale,
+                      double *out) {
+    if (n_kv < 1 || d < 1) return -1;
+    double *z = (double *)malloc((size_t)n_kv * sizeof(double));
+    if (!z) return -1;
+    double zmax = -INFINITY;
+    for (int t = 0; t < n_kv; ++t) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += bf16_to_double(q[c]) * bf16_to_double(k[(size_t)t * d + c]);
+        z[t] = scale * dot;
+        if (z[t] > zmax) zmax = z[t];
+    }
+    double den = 0.0;
+    for (int t = 0; t < n_kv; ++t) {
+        z[t] = exp(z[t] - zmax);
+        den += z[t];
+    }
+    for (int c = 0; c < d; ++c) out[c] = 0.0;
+    for (int t = 0; t < n_kv; ++t) {
+        const double pt = z[t] / den;
+        for (int c = 0; c < d; ++c) out[c] += pt * bf16_to_double(v[(size_t)t * d + c]);
+    }
+    free(z);
+    return 0;
+}

@@ -18,7 +18,7 @@ from .binding import (  # noqa: F401
     SpeckvError, load_library, library_path,
     speckv_workspace_size, speckv_score, speckv_row_lse,
     specpc_workspace_size, specpc_score,
-    topk_workspace_size, topk_select, kv_compact,
+    topk_workspace_size, topk_select, kv_compact, decode_attention,
     spk_device_error, spk_selftest_wait_timeout, spk_exp2_fma, mapped_host_pointer,
 )
 from .pipeline import speckv_compress, specpc_select, cascade_compress  # noqa: F401
@@ -27,7 +27,7 @@ __all__ = [
     "SpeckvError", "load_library", "library_path",
     "speckv_workspace_size", "speckv_score", "speckv_row_lse",
     "specpc_workspace_size", "specpc_score",
-    "topk_workspace_size", "topk_select", "kv_compact",
+    "topk_workspace_size", "topk_select", "kv_compact", "decode_attention",
     "spk_device_error", "spk_selftest_wait_timeout", "spk_exp2_fma", "mapped_host_pointer",
     "speckv_compress", "specpc_select", "cascade_compress",
 ]

@@ -70,6 +70,7 @@ def load_library():
         "spk_selftest_wait_timeout": (I, [ctypes.c_longlong, vp]),
         "spk_exp2_fma": (I, [vp, vp, I, vp]),
         "spk_mapped_host_pointer": (I, [vp, ctypes.POINTER(vp)]),
+        "decode_attention": (I, [I, I, I, I, I, I, F, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -219,6 +220,20 @@ def kv_compact(k, v, idx, k_out, v_out, units_per_idx: int = 1, stream=None):
                           _dev(idx, "idx", torch.int32), n_idx, units_per_idx, _dev(k_out, "k_out"),
                           _dev(v_out, "v_out"), _stream(stream)))
     return k_out, v_out
+
+
+def decode_attention(q, k, v, out=None, scale: float = 1.0, stream=None):
+    """Decode attention over a compacted cache: q [B, L, Hq, d], k/v [B, L, Hkv, n_kv, d]
+    (bf16, CUDA) -> out fp32 [B, L, Hq, d]."""
+    lib = load_library()
+    Bsz, L, hq, d = q.shape
+    hkv, n_kv = k.shape[2], k.shape[3]
+    if out is None:
+        out = torch.empty((Bsz, L, hq, d), dtype=torch.float32, device=q.device)
+    _check(lib.decode_attention(Bsz, L, hq, hkv, d, n_kv, float(scale), _dev(q, "q", torch.bfloat16),
+                                _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+                                _dev(out, "out", torch.float32), _stream(stream)))
+    return out
 
 
 # --------------------------------------------------------------------- errors

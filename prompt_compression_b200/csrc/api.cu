@@ -15,6 +15,10 @@
 #include "score.cuh"
 
 namespace spk {
+// decode.cu
+cudaError_t launch_decode(const void* q, const void* k, const void* v, float* out, int units, int g,
+                          int head_dim, int n_kv, float c2, cudaStream_t stream);
+
 namespace {
 
 thread_local char g_msg[512] = "";
@@ -328,6 +332,29 @@ spk_status kv_compact(const void* k, const void* v, int units, int n_src, int he
 }
 
 // ------------------------------------------------------------------ device errors
+// ------------------------------------------------------------------ decode
+spk_status decode_attention(int batch, int layers, int hq, int hkv, int head_dim, int n_kv, float scale,
+                            const void* q, const void* k, const void* v, float* out, void* stream) {
+  if (batch < 1 || layers < 1 || hq < 1 || hkv < 1 || n_kv < 1)
+    return fail(SPK_ERR_ARG, "batch, layers, hq, hkv and n_kv must be >= 1");
+  if (hq % hkv != 0) return fail(SPK_ERR_ARG, "hq (%d) must be a multiple of hkv (%d)", hq, hkv);
+  if (hq / hkv > 8) return fail(SPK_ERR_UNSUPPORTED, "hq / hkv = %d exceeds 8", hq / hkv);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(SPK_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+  if (!(scale > 0.f) || !std::isfinite(scale)) return fail(SPK_ERR_ARG, "scale must be finite and > 0");
+  const long long units = static_cast<long long>(batch) * layers * hkv;
+  if (units > 0x7fffffffLL || static_cast<long long>(n_kv) * head_dim > (1LL << 40) / units)
+    return fail(SPK_ERR_UNSUPPORTED, "too many units or rows");
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr)
+    return fail(SPK_ERR_ARG, "q, k, v and out must be non-NULL device pointers");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SPK_ERR_ARG, "q, k, v and out must be 16-byte aligned");
+  cudaError_t e = launch_decode(q, k, v, out, static_cast<int>(units), hq / hkv, head_dim, n_kv,
+                                scale * 1.4426950408889634f, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  return ok();
+}
+
 spk_status spk_mapped_host_pointer(const void* host, void** dev) {
   if (host == nullptr || dev == nullptr) return fail(SPK_ERR_ARG, "host and dev must be non-NULL");
   void* d = nullptr;

@@ -103,3 +103,18 @@ def test_mapped_host_pointer_rejects_unmapped_memory(lib):
     assert rc != 0
     assert out.value == 12345
     assert lib.spk_mapped_host_pointer(None, ctypes.byref(out)) == 1   # SPK_ERR_ARG
+
+
+@pytest.mark.parametrize("args,status,needle", [
+    ((1, 1, 4, 3, 128, 10, 1.0), 1, "multiple"),
+    ((1, 1, 36, 2, 128, 10, 1.0), 2, "exceeds 8"),
+    ((1, 1, 4, 2, 96, 10, 1.0), 2, "head_dim"),
+    ((1, 1, 4, 2, 128, 0, 1.0), 1, ">= 1"),
+    ((1, 1, 4, 2, 128, 10, -1.0), 1, "scale"),
+    ((1, 1, 4, 2, 128, 10, 1.0), 1, "non-NULL"),
+])
+def test_decode_argument_errors(lib, args, status, needle):
+    B, L, hq, hkv, d, n_kv, scale = args
+    rc = lib.decode_attention(B, L, hq, hkv, d, n_kv, ctypes.c_float(scale), None, None, None, None, None)
+    assert rc == status
+    assert needle in lib.spk_last_error().decode()

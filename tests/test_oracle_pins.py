@@ -323,3 +323,73 @@ def test_tiny_workload_recovers_planted_keys():
         sel = set(idx.tolist())
         assert {0, 100, 101, 102, 103} <= sel      # sink and heavy keys are kept
         assert s[0] > np.quantile(s, 0.9)            # the sink ranks high
+
+
+# ---------------------------------------------------------------- decode attention
+def _bf(x):
+    return W.bf16_bits(np.asarray(x, np.float32))
+
+
+def test_decode_single_row_returns_its_value():
+    rng = np.random.default_rng(31)
+    q = _bf(rng.standard_normal((1, 1, 2, 64)))
+    k = _bf(rng.standard_normal((1, 1, 1, 1, 64)))
+    v = _bf(rng.standard_normal((1, 1, 1, 1, 64)))
+    out = oracle.decode_attention(q, k, v, 0.3)
+    np.testing.assert_array_equal(out[0, 0, 0], W.bf16_decode(v)[0, 0, 0, 0].astype(np.float64))
+    np.testing.assert_array_equal(out[0, 0, 1], W.bf16_decode(v)[0, 0, 0, 0].astype(np.float64))
+
+
+def test_decode_identical_keys_average_the_values():
+    rng = np.random.default_rng(32)
+    q = _bf(rng.standard_normal((1, 1, 1, 64)))
+    k = _bf(np.tile(rng.standard_normal((1, 1, 1, 1, 64)), (1, 1, 1, 9, 1)))
+    v = _bf(rng.standard_normal((1, 1, 1, 9, 64)))
+    out = oracle.decode_attention(q, k, v, 1.0)
+    np.testing.assert_allclose(out[0, 0, 0], W.bf16_decode(v)[0, 0, 0].astype(np.float64).mean(0), rtol=0, atol=1e-14)
+
+
+def test_decode_two_keys_closed_form():
+    # z_i = scale * a * b_i exactly (one nonzero coordinate, bf16-exact numbers):
+    # out = sigma(z_0 - z_1) v_0 + sigma(z_1 - z_0) v_1
+    d = 64
+    q = np.zeros((1, 1, 1, d), np.float32); q[..., 5] = 1.5
+    k = np.zeros((1, 1, 1, 2, d), np.float32); k[..., 0, 5] = 2.0; k[..., 1, 5] = -0.75
+    v = np.zeros((1, 1, 1, 2, d), np.float32); v[..., 0, :] = 3.0; v[..., 1, :] = -1.0
+    scale = 0.5
+    out = oracle.decode_attention(_bf(q), _bf(k), _bf(v), scale)
+    z0, z1 = scale * 1.5 * 2.0, scale * 1.5 * -0.75
+    p0 = 1.0 / (1.0 + math.exp(z1 - z0))
+    np.testing.assert_allclose(out[0, 0, 0], np.full(d, 3.0 * p0 - (1.0 - p0)), rtol=1e-14)
+
+
+def test_decode_gqa_heads_read_their_kv_head():
+    # KV head 0 holds values +1, KV head 1 values -1: query heads 0, 1 -> +1 and 2, 3 -> -1
+    rng = np.random.default_rng(33)
+    q = _bf(rng.standard_normal((1, 1, 4, 64)))
+    k = _bf(rng.standard_normal((1, 1, 2, 7, 64)))
+    v = np.ones((1, 1, 2, 7, 64), np.float32); v[:, :, 1] = -1.0
+    out = oracle.decode_attention(q, k, _bf(v), 0.2)
+    np.testing.assert_allclose(out[0, 0, :2], 1.0, rtol=1e-14)
+    np.testing.assert_allclose(out[0, 0, 2:], -1.0, rtol=1e-14)
+
+
+def test_decode_row_order_does_not_matter():
+    rng = np.random.default_rng(34)
+    q = _bf(rng.standard_normal((1, 2, 3, 128)))
+    k = _bf(rng.standard_normal((1, 2, 1, 40, 128)))
+    v = _bf(rng.standard_normal((1, 2, 1, 40, 128)))
+    perm = rng.permutation(40)
+    a = oracle.decode_attention(q, k, v, 0.09)
+    b = oracle.decode_attention(q, k[:, :, :, perm], v[:, :, :, perm], 0.09)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+def test_decode_dominant_key_wins():
+    d = 64
+    q = np.zeros((1, 1, 1, d), np.float32); q[..., 0] = 8.0
+    k = np.zeros((1, 1, 1, 5, d), np.float32); k[..., 3, 0] = 8.0          # logit 64 vs 0
+    v = np.arange(5 * d, dtype=np.float32).reshape(1, 1, 1, 5, d) / 64.0
+    out = oracle.decode_attention(_bf(q), _bf(k), _bf(v), 1.0)
+    # the other four rows carry weight e^-64 each, |v| <= 5
+    np.testing.assert_allclose(out[0, 0, 0], W.bf16_decode(_bf(v))[0, 0, 0, 3], rtol=0, atol=4 * 10 * math.exp(-64))

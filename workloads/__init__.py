@@ -131,6 +131,25 @@ class CascadeConfig:
     n_in_full: int                # tokens before the SpecPC gather
 
 
+@dataclasses.dataclass(frozen=True)
+class DecodeConfig:
+    """One decode step (one new query token per head) over the cache that
+    SpecKV leaves (section "整体框架": the target then runs on the compressed
+    cache), and, for contrast, over the full cache."""
+    name: str
+    batch: int
+    layers: int
+    hq: int
+    hkv: int
+    head_dim: int
+    n_kv: int                     # kept rows per KV head (C_max + n_window)
+    n_kv_full: int                # rows of the uncompressed cache
+
+    @property
+    def units(self) -> int:
+        return self.batch * self.layers * self.hkv
+
+
 TINY = SpecKVConfig("tiny_speckv", batch=1, layers=1, hq=4, hkv=2, head_dim=64,
                     n_in=512, n_window=16, n_lookahead=16, c_max=64, pool=7)
 LLAMA8B_16K = SpecKVConfig("llama3.1-8b_speckv_16k", batch=1, layers=32, hq=32, hkv=8,
@@ -150,7 +169,11 @@ CASCADE_128K = CascadeConfig(
                         n_in=2048, n_window=64, n_lookahead=64, c_max=256, heavy_frac=0.01),
     n_in_full=131072)
 
-CONFIGS = {c.name: c for c in (TINY, LLAMA8B_16K, QWEN32B_64K, QWEN05B_SPECPC_32K, CASCADE_128K)}
+DECODE_QWEN32B = DecodeConfig("qwen2.5-32b_decode_compressed", batch=1, layers=64, hq=40, hkv=8,
+                              head_dim=128, n_kv=320, n_kv_full=65536)
+
+CONFIGS = {c.name: c for c in (TINY, LLAMA8B_16K, QWEN32B_64K, QWEN05B_SPECPC_32K, CASCADE_128K,
+                               DECODE_QWEN32B)}
 
 
 # ---------------------------------------------------------------------------
