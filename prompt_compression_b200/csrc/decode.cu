@@ -9,15 +9,17 @@
 // over the n_kv rows of the head's KV head (GQA: query head qh reads KV head
 // qh / g), e.g. the k_out / v_out that kv_compact leaves.
 //
-// One CTA (8 warps) per (batch, layer, KV head) unit.  Warp w takes rows
-// t = 4w.., in blocks of 4 rows every 32 (so each block's K and V rows are
-// independent loads in flight together); lane l holds elements
-// [l * d/32, (l + 1) * d/32) of every row, so a row is one coalesced 128- or
-// 256-byte load.  For each of the g query heads the warp keeps an online
-// softmax state (running max in the log2 domain, running sum, and its lanes'
-// slice of the weighted V sum).  At the end the 8 warps' states are merged
-// in a fixed order, so results are bitwise reproducible.  Every K and V byte
-// is read once: the kernel is bound by HBM bandwidth.
+// One CTA (8 warps) per (batch, layer, KV head) unit; warp w takes the
+// 32-row blocks w, w + 8, ...  Within a block, lane l owns row t0 + l for the
+// logits: it reads its K row in 16-byte pieces and dots it with the g query
+// rows held in shared memory (broadcast reads), so no cross-lane reduction
+// is needed per row.  The block's max and sum per query head take one warp
+// reduction each (online softmax: log2-domain running max and sum), the
+// weights go to shared memory, and for the weighted V sum lane l owns
+// elements [l * d/32, (l + 1) * d/32) of every V row (coalesced row loads).
+// At the end the 8 warps' states are merged in a fixed order, so results
+// are bitwise reproducible.  Every K and V byte is read once: the kernel is
+// bound by HBM bandwidth.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -27,7 +29,6 @@ namespace spk {
 namespace {
 
 constexpr int kDecWarps = 8;
-constexpr int kDecRowsPerIter = 4;   // rows a warp has in flight per iteration
 
 template <int D>
 struct RowSlice;   // one lane's d/32 bf16 elements of a row
@@ -63,20 +64,18 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
                   float* __restrict__ out, int n_kv, float c2) {
   using S = RowSlice<D>;
-  constexpr int E = S::kN;
+  constexpr int E = S::kN;   // V elements per lane
+  __shared__ __align__(16) float q_s[G][D];
+  __shared__ float p_s[kDecWarps][G][32];
   __shared__ float m_s[kDecWarps][G], l_s[kDecWarps][G];
   __shared__ float acc_s[kDecWarps][G][D];
 
-  const int unit = blockIdx.x;   // (b * layers + l) * hkv + h
+  const int unit = blockIdx.x;   // (b * layers + l) * hkv + h; its query heads are rows unit*G .. unit*G+G-1
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // this unit's query heads are G consecutive rows of q: unit * G .. unit * G + G - 1
-  float qf[G][E];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const typename S::T r =
-        reinterpret_cast<const typename S::T*>(q + (static_cast<size_t>(unit) * G + h) * D)[lane];
-    unpack<D>(r, qf[h]);
-  }
+  for (int i = threadIdx.x; i < G * D; i += kDecWarps * 32)
+    q_s[i / D][i % D] = __uint_as_float(static_cast<uint32_t>(q[static_cast<size_t>(unit) * G * D + i]) << 16);
+  __syncthreads();
+
   float m[G], l[G], acc[G][E];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -85,41 +84,70 @@ __global__ void __launch_bounds__(kDecWarps * 32)
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
   }
-  const typename S::T* kr = reinterpret_cast<const typename S::T*>(k + static_cast<size_t>(unit) * n_kv * D);
+  const uint16_t* kr = k + static_cast<size_t>(unit) * n_kv * D;
   const typename S::T* vr = reinterpret_cast<const typename S::T*>(v + static_cast<size_t>(unit) * n_kv * D);
 
-  for (int t0 = warp * kDecRowsPerIter; t0 < n_kv; t0 += kDecWarps * kDecRowsPerIter) {
-    typename S::T kv_k[kDecRowsPerIter], kv_v[kDecRowsPerIter];
+  for (int t0 = warp * 32; t0 < n_kv; t0 += kDecWarps * 32) {
+    const int t = t0 + lane;
+    const bool valid = t < n_kv;
+    // logits of this lane's row for every query head of the group
+    const uint4* krow = reinterpret_cast<const uint4*>(kr + static_cast<size_t>(valid ? t : t0) * D);
+    float z[G];
 #pragma unroll
-    for (int i = 0; i < kDecRowsPerIter; ++i) {
-      const int t = t0 + i < n_kv ? t0 + i : t0;   // rows past the end repeat a valid row (masked below)
-      kv_k[i] = __ldcs(kr + static_cast<size_t>(t) * 32 + lane);
-      kv_v[i] = __ldcs(vr + static_cast<size_t>(t) * 32 + lane);
-    }
-#pragma unroll
-    for (int i = 0; i < kDecRowsPerIter; ++i) {
-      float kf[E], vf[E];
-      unpack<D>(kv_k[i], kf);
-      unpack<D>(kv_v[i], vf);
-      const bool valid = t0 + i < n_kv;
+    for (int h = 0; h < G; ++h) z[h] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 kk = __ldg(krow + c);
+      const float kf[8] = {bf16_lo(kk.x), bf16_hi(kk.x), bf16_lo(kk.y), bf16_hi(kk.y),
+                           bf16_lo(kk.z), bf16_hi(kk.z), bf16_lo(kk.w), bf16_hi(kk.w)};
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float s = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) s = fmaf(qf[h][e], kf[e], s);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (!valid) continue;
-        const float z = s * c2;                       // log2-domain logit
-        const float mn = fmaxf(m[h], z);
-        const float alpha = ex2_approx(m[h] - mn);    // 0 on the first row (m = -inf)
-        const float pz = ex2_approx(z - mn);
-        l[h] = l[h] * alpha + pz;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[h][e] = fmaf(acc[h][e], alpha, pz * vf[e]);
-        m[h] = mn;
+        const float4 qa = *reinterpret_cast<const float4*>(&q_s[h][c * 8]);
+        const float4 qb = *reinterpret_cast<const float4*>(&q_s[h][c * 8 + 4]);
+        z[h] = fmaf(qa.x, kf[0], z[h]);
+        z[h] = fmaf(qa.y, kf[1], z[h]);
+        z[h] = fmaf(qa.z, kf[2], z[h]);
+        z[h] = fmaf(qa.w, kf[3], z[h]);
+        z[h] = fmaf(qb.x, kf[4], z[h]);
+        z[h] = fmaf(qb.y, kf[5], z[h]);
+        z[h] = fmaf(qb.z, kf[6], z[h]);
+        z[h] = fmaf(qb.w, kf[7], z[h]);
       }
     }
+    // online softmax over the block, per query head
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float zz = valid ? z[h] * c2 : -INFINITY;   // log2-domain logit
+      float bm = zz;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+      const float mn = fmaxf(m[h], bm);
+      const float alpha = ex2_approx(m[h] - mn);   // 0 while m = -inf
+      const float pz = valid ? ex2_approx(zz - mn) : 0.f;
+      float bs = pz;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bs += __shfl_xor_sync(0xffffffffu, bs, o);
+      l[h] = fmaf(l[h], alpha, bs);
+      m[h] = mn;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[h][e] *= alpha;
+      p_s[warp][h][lane] = pz;
+    }
+    __syncwarp();
+    // weighted V sum over the block's rows; lane owns E elements of a row
+    const int rows = n_kv - t0 < 32 ? n_kv - t0 : 32;
+#pragma unroll 2
+    for (int j = 0; j < rows; ++j) {
+      float vf[E];
+      unpack<D>(__ldcs(vr + static_cast<size_t>(t0 + j) * 32 + lane), vf);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float pj = p_s[warp][h][j];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[h][e] = fmaf(pj, vf[e], acc[h][e]);
+      }
+    }
+    __syncwarp();
   }
   // merge the warps' states in a fixed order
 #pragma unroll
