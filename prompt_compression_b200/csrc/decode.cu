@@ -95,9 +95,12 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     float z[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) z[h] = 0.f;
-#pragma unroll 2
+    uint4 kbuf[D / 8];   // the whole row in flight at once
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) kbuf[c] = __ldg(krow + c);
+#pragma unroll
     for (int c = 0; c < D / 8; ++c) {
-      const uint4 kk = __ldg(krow + c);
+      const uint4 kk = kbuf[c];
       const float kf[8] = {bf16_lo(kk.x), bf16_hi(kk.x), bf16_lo(kk.y), bf16_hi(kk.y),
                            bf16_lo(kk.z), bf16_hi(kk.z), bf16_lo(kk.w), bf16_hi(kk.w)};
 #pragma unroll
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     __syncwarp();
     // weighted V sum over the block's rows; lane owns E elements of a row
     const int rows = n_kv - t0 < 32 ? n_kv - t0 : 32;
-#pragma unroll 2
+#pragma unroll 4
     for (int j = 0; j < rows; ++j) {
       float vf[E];
       unpack<D>(__ldcs(vr + static_cast<size_t>(t0 + j) * 32 + lane), vf);
