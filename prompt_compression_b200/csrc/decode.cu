@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     __syncwarp();
     // weighted V sum over the block's rows; lane owns E elements of a row
     const int rows = n_kv - t0 < 32 ? n_kv - t0 : 32;
-#pragma unroll 4
+#pragma unroll 8
     for (int j = 0; j < rows; ++j) {
       float vf[E];
       unpack<D>(__ldcs(vr + static_cast<size_t>(t0 + j) * 32 + lane), vf);
