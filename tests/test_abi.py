@@ -118,3 +118,28 @@ def test_decode_argument_errors(lib, args, status, needle):
     rc = lib.decode_attention(B, L, hq, hkv, d, n_kv, ctypes.c_float(scale), None, None, None, None, None)
     assert rc == status
     assert needle in lib.spk_last_error().decode()
+
+
+def _prototypes():
+    """name -> number of parameters, from the header's declarations."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"\b([a-z_][a-z0-9_]*)\s*\(([^;{}]*?)\)\s*;", text, flags=re.S):
+        name, params = m.group(1), m.group(2).strip()
+        protos[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_signatures_match_the_header(lib):
+    # every function the Python binding declares takes as many arguments as
+    # its prototype in include/speckv.h (the boundary cannot drift silently)
+    protos = _prototypes()
+    checked = 0
+    for name, n in protos.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == n, f"{name}: header has {n} parameters, binding {len(fn.argtypes)}"
+        checked += 1
+    assert checked >= 10
