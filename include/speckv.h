@@ -181,7 +181,9 @@ spk_status topk_select(const float* scores, int units, int n_cand, int pool_kern
  * layers * hkv shares one row across all (layer, KV head) of a batch element
  * (SpecPC / SpecKV-PC).  v and v_out may both be NULL.  Rows are copied
  * byte for byte.  An index outside [0, n_src) leaves that output row
- * unwritten and records SPK_ERR_ARG in the device error word.
+ * unwritten and records SPK_ERR_ARG in the device error word.  k and v may
+ * be device addresses of pinned host memory (spk_mapped_host_pointer): only
+ * the selected rows are then read over the host link.
  *
  * Supported: head_dim * elem_bytes a multiple of 16; units % units_per_idx == 0.
  * ------------------------------------------------------------------------ */
