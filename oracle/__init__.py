@@ -50,11 +50,12 @@ def _load():
         lib.oracle_specpc_batch.argtypes = [_u16p, _u16p, _dp, I, I, I, I, I, I, I, I, D, _dp]
         lib.oracle_specpc_batch_f64.argtypes = [_dp, _dp, _dp, I, I, I, I, I, I, I, I, D, _dp]
         lib.oracle_maxpool.argtypes = [_dp, I, I, _dp]
+        lib.oracle_avgpool.argtypes = [_dp, I, I, _dp]
         lib.oracle_topk_with_tail.argtypes = [_dp, I, I, I, _i32p]
         lib.oracle_gather_rows.argtypes = [_u8p, I, I, _i32p, I, _u8p]
         lib.oracle_decode_row.argtypes = [_u16p, _u16p, _u16p, I, I, D, _dp]
         for f in (lib.oracle_speckv_unit, lib.oracle_speckv_unit_f64, lib.oracle_specpc_batch,
-                  lib.oracle_specpc_batch_f64, lib.oracle_maxpool, lib.oracle_topk_with_tail,
+                  lib.oracle_specpc_batch_f64, lib.oracle_maxpool, lib.oracle_avgpool, lib.oracle_topk_with_tail,
                   lib.oracle_gather_rows, lib.oracle_decode_row):
             f.restype = ctypes.c_int
         _lib = lib
@@ -131,6 +132,20 @@ def maxpool(s, kernel: int = 7):
     out = np.zeros_like(s)
     _check(lib.oracle_maxpool(_ptr(s, _dp), s.size, kernel, _ptr(out, _dp)))
     return out
+
+
+def avgpool(s, kernel: int = 7):
+    """Mean over the window [j - r, j + r] clipped to the row, r = kernel // 2."""
+    lib = _load()
+    s = np.ascontiguousarray(s, np.float64)
+    out = np.zeros_like(s)
+    _check(lib.oracle_avgpool(_ptr(s, _dp), s.size, kernel, _ptr(out, _dp)))
+    return out
+
+
+def pool(s, kernel: int = 7, mode: str = "max"):
+    """Local pooling of one row of scores: mode "max" or "avg"."""
+    return maxpool(s, kernel) if mode == "max" else avgpool(s, kernel)
 
 
 def topk_with_tail(pooled, k: int, n_tail: int):

@@ -26,7 +26,9 @@
  *     the window is kept unconditionally;
  *   - the GQA group of KV head h is query heads h*g .. h*g+g-1, and their
  *     attention is summed; rows are summed without weights;
- *   - pooling is a stride-1 max over the clipped window [j-r, j+r];
+ *   - pooling is a stride-1 max (or, as the averaging variant, the mean)
+ *     over the window [j-r, j+r] clipped to the row;
+ *   - a SpecPC row of weight 0 contributes nothing;
  *   - ties in the selection go to the lower index; the output lists the
  *     selected indices in ascending order, then the window.
  *
@@ -203,6 +205,24 @@ int oracle_maxpool(const double *s, int n, int kernel, double *out) {
         for (int t = lo + 1; t <= hi; ++t)
             if (s[t] > m) m = s[t];
         out[j] = m;
+    }
+    return 0;
+}
+
+/*
+ * 1-D average pooling, odd kernel, stride 1, output length n: the mean of the
+ * scores inside the window clipped at the row's ends (the pages name local
+ * pooling without its kind; this is the averaging reading of it).
+ */
+int oracle_avgpool(const double *s, int n, int kernel, double *out) {
+    if (kernel < 1 || (kernel & 1) == 0 || n < 0) return -1;
+    const int r = kernel / 2;
+    for (int j = 0; j < n; ++j) {
+        int lo = j - r < 0 ? 0 : j - r;
+        int hi = j + r > n - 1 ? n - 1 : j + r;
+        double sum = 0.0;
+        for (int t = lo; t <= hi; ++t) sum += s[t];
+        out[j] = sum / (double)(hi - lo + 1);
     }
     return 0;
 }

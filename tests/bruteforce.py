@@ -4,13 +4,13 @@ These materialise what the pages describe literally -- the full causal
 attention matrix of every query row (SpecKV), or the draft attention tensor
 A[layer][head][query position][key] over all query positions (SpecPC) --
 and reduce it with library routines (scipy.special.softmax,
-scipy.ndimage.maximum_filter1d, numpy.lexsort).  They are written
+scipy.ndimage.maximum_filter1d / uniform_filter1d, numpy.lexsort).  They are written
 independently of oracle.c and only for tiny inputs.
 """
 from __future__ import annotations
 
 import numpy as np
-from scipy.ndimage import maximum_filter1d
+from scipy.ndimage import maximum_filter1d, uniform_filter1d
 from scipy.special import softmax
 
 
@@ -66,6 +66,16 @@ def specpc_batch(q_all, k, weights, l_skip, scale=1.0):
 def maxpool(s, kernel):
     # 'nearest' edge replication gives the same maximum as clipping the window
     return maximum_filter1d(np.asarray(s, np.float64), size=kernel, mode="nearest")
+
+
+def avgpool(s, kernel):
+    """Mean over the clipped window: a zero-padded box sum over a zero-padded
+    box count (two uniform filters with constant-0 edges, whose 1/kernel
+    factors cancel)."""
+    s = np.asarray(s, np.float64)
+    num = uniform_filter1d(s, size=kernel, mode="constant", cval=0.0)
+    den = uniform_filter1d(np.ones_like(s), size=kernel, mode="constant", cval=0.0)
+    return num / den
 
 
 def topk_with_tail(pooled, k, n_tail):

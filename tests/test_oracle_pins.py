@@ -191,6 +191,30 @@ def test_maxpool_plateau_by_hand():
     assert oracle.maxpool(s, 7).tolist() == [5.0] * 7 + [0.0] * 4
 
 
+@pytest.mark.parametrize("kernel", [1, 3, 7, 9, 31])
+def test_avgpool_matches_library_filters(kernel):
+    # the average over the window clipped to the row: a library box filter
+    # with zero padding, divided by the same filter applied to ones
+    rng = np.random.default_rng(kernel)
+    for n in (1, 2, 5, 40, 333):
+        s = rng.random(n)
+        np.testing.assert_allclose(oracle.avgpool(s, kernel), bf.avgpool(s, kernel), rtol=1e-13, atol=0)
+
+
+def test_avgpool_by_hand():
+    # kernel 3 on (0, 3, 6, 9): ends average two values, the middle three
+    assert oracle.avgpool(np.array([0.0, 3.0, 6.0, 9.0]), 3).tolist() == [1.5, 3.0, 6.0, 7.5]
+    # a kernel wider than the row averages the whole row everywhere
+    assert oracle.avgpool(np.array([1.0, 2.0, 6.0]), 9).tolist() == [3.0, 3.0, 3.0]
+    assert oracle.pool(np.array([1.0, 5.0, 2.0]), 3, "avg").tolist() == [3.0, 8.0 / 3.0, 3.5]
+    assert oracle.pool(np.array([1.0, 5.0, 2.0]), 3, "max").tolist() == [5.0, 5.0, 5.0]
+
+
+def test_avgpool_rejects_even_kernel():
+    with pytest.raises(ValueError):
+        oracle.avgpool(np.zeros(5), 2)
+
+
 def test_maxpool_rejects_even_kernel():
     with pytest.raises(ValueError):
         oracle.maxpool(np.zeros(5), 4)
@@ -228,6 +252,48 @@ def test_specpc_matches_full_attention_tensor(L, l_skip, hq, hkv, n_in, n_lookah
     got = oracle.specpc_batch(q_all[:, :, T - Wr:], k, w, l_skip, n_lookahead)
     ref = bf.specpc_batch(q_all, k, w, l_skip)
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-16)
+
+
+@pytest.mark.parametrize("L,l_skip,hq,hkv,n_in,n_lookahead,Wr,d", [
+    (3, 1, 4, 2, 40, 1, 8, 8),     # every dimension distinct from the others
+    (2, 0, 6, 3, 23, 3, 5, 16),
+    (4, 2, 2, 1, 17, 1, 16, 4),    # W close to n_in
+])
+def test_specpc_bf16_entry_matches_bruteforce_on_decoded_values(L, l_skip, hq, hkv, n_in, n_lookahead, Wr, d):
+    # The bf16 entry decodes q [L][Hq][W][d] and k [L][Hkv][n_in][d] itself;
+    # it must equal the float entry on the decoded values exactly and the
+    # brute-force draft attention tensor built from those values.  A size,
+    # offset or tensor mix-up in the decode (say, q's element count used for
+    # k) changes these numbers.
+    rng = np.random.default_rng(L * 1000 + n_in * 10 + d)
+    T = n_in + n_lookahead - 1
+    q_all = W.bf16_bits((rng.standard_normal((L, hq, T, d)) / math.sqrt(d)).astype(np.float32))
+    kb = W.bf16_bits(rng.standard_normal((L, hkv, n_in, d)).astype(np.float32))
+    qb = np.ascontiguousarray(q_all[:, :, T - Wr:])
+    w = W.specpc_row_weights(Wr)
+    got = oracle.specpc_batch(qb, kb, w, l_skip, n_lookahead)
+    f64 = oracle.specpc_batch(W.bf16_decode(qb).astype(np.float64), W.bf16_decode(kb).astype(np.float64),
+                              w, l_skip, n_lookahead)
+    assert np.array_equal(got, f64)
+    ref = bf.specpc_batch(W.bf16_decode(q_all).astype(np.float64), W.bf16_decode(kb).astype(np.float64), w, l_skip)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-16)
+
+
+def test_specpc_zero_weight_rows_contribute_nothing():
+    # rows of weight 0 drop out of the weighted mean: the brute-force
+    # attention tensor with the same weights, and, where only the zero-weight
+    # (latest) rows see a key, a score of exactly 0
+    rng = np.random.default_rng(31)
+    L, hq, hkv, n_in, nl, Wr, d = 2, 4, 2, 30, 1, 6, 8
+    T = n_in + nl - 1
+    q_all = rng.standard_normal((L, hq, T, d)) / math.sqrt(d)
+    k = rng.standard_normal((L, hkv, n_in, d))
+    w = np.array([0.3, 0.0, 1.0, 0.5, 0.0, 0.0])
+    got = oracle.specpc_batch(q_all[:, :, T - Wr:], k, w, 0, nl)
+    np.testing.assert_allclose(got, bf.specpc_batch(q_all, k, w, 0), rtol=1e-12, atol=1e-16)
+    # the last two rows (positions n_in-2, n_in-1) have weight 0 and are the
+    # only rows that see keys n_in-2 and n_in-1; row 3 (weight 0.5) sees n_in-3
+    assert got[n_in - 1] == 0.0 and got[n_in - 2] == 0.0 and got[n_in - 3] > 0.0
 
 
 def test_specpc_single_row_is_softmax():
