@@ -2,23 +2,28 @@
 """Throughput of the lookahead importance-scoring path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--cmax C]
+    python bench.py --suite ...               # one JSON line per workload
     python bench.py --impl reference ...      # the fp64 CPU oracle on the host cores
 
-One step = speckv_score (row-LSE pass + column-sum pass) + topk_select (pool 7,
-top-C_max + window) + kv_compact over every unit of the workload, through the
-C ABI of libspeckv.so.  Default workload: the Qwen2.5-32B-shaped SpecKV pass at
-64K context (64 layers, 40/8 heads, head_dim 128, window 64, lookahead 128,
+One step = the two scoring passes (speckv_row_offsets + speckv_colsum, which
+together are speckv_score) + topk_select (pool 7, top-C_max + window) +
+kv_compact over every unit of the workload, through the C ABI of
+libspeckv.so.  Default workload: the Qwen2.5-32B-shaped SpecKV pass at 64K
+context (64 layers, 40/8 heads, head_dim 128, window 64, lookahead 128,
 C_max 256), seeded synthetic bf16 inputs resident in HBM (K and V are 8.6 GB
 each, far larger than the 126 MB L2, so no L2 flush is needed between steps).
+CUDA events are recorded on the launching stream between the kernels of
+every timed step, so each kernel's time is measured inside the timed region
+and the kernels' times add up to the step.
 Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
 seed (units are independent, no data-path collective): weak scaling.
-Prints one JSON line on rank 0.
+Prints one JSON line on rank 0 (one per workload with --suite).
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -33,9 +38,12 @@ import numpy as np  # noqa: E402
 import workloads as W  # noqa: E402
 
 METRIC = "KV-head-tokens scored+selected+compacted/s at 64K ctx"
+SUITE = ("llama3.1-8b_speckv_16k", "qwen2.5-32b_speckv_64k", "qwen2.5-32b_speckv_64k@1024",
+         "qwen2.5-32b_speckv_64k@2048", "qwen2.5-0.5b_specpc_32k", "cascade_specpc_speckv_128k",
+         "qwen2.5-32b_decode_compressed")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -43,23 +51,27 @@ def parse():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--config", default=W.QWEN32B_64K.name, choices=list(W.CONFIGS))
     ap.add_argument("--cmax", type=int, default=None)
+    ap.add_argument("--suite", action="store_true", help="one line per workload (headline included)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="e2e: groups of (batch, layer) whose host-to-device copy overlaps the previous group's work")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
-def config_of(args):
-    import dataclasses
-    cfg = W.CONFIGS[args.config]
-    if args.cmax is not None and isinstance(cfg, W.SpecKVConfig):
-        cfg = dataclasses.replace(cfg, c_max=args.cmax)
+def config_of(name, cmax=None):
+    if "@" in name:
+        name, c = name.split("@")
+        cmax = int(c)
+    cfg = W.CONFIGS[name]
+    if cmax is not None and isinstance(cfg, W.SpecKVConfig):
+        cfg = dataclasses.replace(cfg, c_max=cmax)
     return cfg
 
 
+# ----------------------------------------------------------------- work and bytes
 def specpc_flops(cfg: W.SpecPCConfig) -> float:
     """One Q.K^T product over the causally visible keys of every SpecPC row
     (query position n_in + n_lookahead - 1 - W + i), all query heads and
@@ -84,6 +96,11 @@ def algorithmic_bytes(cfg: W.SpecKVConfig) -> float:
     return per_unit * cfg.units
 
 
+def topk_bytes(units: int, n_cand: int, out_len: int) -> float:
+    """The selection's algorithmic traffic: every score read once, the indices written."""
+    return units * (4.0 * n_cand + 4.0 * out_len)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -94,6 +111,21 @@ def load_peaks():
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "source": "fallback"}
+
+
+def tensor_peak(peaks):
+    """Every kernel is timed per launch (milliseconds each): the roofline
+    denominator is the burst bf16 GEMM figure.  The sustained (power-capped,
+    seconds-long) figure is reported beside it for context only."""
+    return peaks["bf16_tflops"], f"{peaks['source']} bf16 burst (per-launch kernel timing)"
+
+
+def exp2_peak_per_s():
+    """Exponentials per second the SMs can produce: the MUFU gives 16 ex2 per
+    clock per SM; the FMA pipe (128 lanes) spends 2 lane-ops per logit on the
+    scale and the sum and 7 per polynomial exponential, so the best split
+    (40 % polynomial) reaches 16 / 0.6 = 26.7 exponentials per clock per SM."""
+    return 148 * (16.0 / 0.6) * 1965e6
 
 
 # ----------------------------------------------------------------- clocks
@@ -149,76 +181,44 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# ----------------------------------------------------------------- oracle timing
-def _oracle_unit_job(payload):
-    """Scores -> pool -> top-C_max + window -> gather, for one unit (fp64 oracle)."""
-    sys.path.insert(0, ROOT)
-    import oracle
-    qb, kb, vb, n_window, n_lookahead, c_max, pool = payload
-    s, p, idx = oracle.speckv_select_unit(qb, kb, n_window, n_lookahead, c_max, pool)
-    oracle.gather_rows(kb, idx)
-    oracle.gather_rows(vb, idx)
-    return int(idx.size)
+# ----------------------------------------------------------------- timed steps
+def timed_steps(launches, steps, warmup, stream, barrier=lambda: None):
+    """Run `warmup` untimed steps, then `steps` timed ones.  A step runs the
+    (name, fn) launches in order; a CUDA event is recorded on `stream` before
+    the first launch and after every launch.  Returns the total device time
+    of the timed steps (first event to last), each launch's mean time, the
+    median step time and the clock summary sampled during the timed steps."""
+    import torch
+    for _ in range(warmup):
+        for _, fn in launches:
+            fn()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(launches) + 1)] for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        time.sleep(0.3)
+        for s in range(steps):
+            ev[s][0].record(stream)
+            for i, (_, fn) in enumerate(launches):
+                fn()
+                ev[s][i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total = ev[0][0].elapsed_time(ev[-1][-1])
+    per = {name: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps
+           for i, (name, _) in enumerate(launches)}
+    step_ms = sorted(ev[s][0].elapsed_time(ev[s][-1]) for s in range(steps))
+    return total, per, step_ms[len(step_ms) // 2], clk.summary()
 
 
-def tensor_peak(peaks):
-    """The scoring kernels run back to back for the whole timed region (tens of
-    milliseconds per step, many steps), under the board power cap: the roofline
-    denominator is the sustained bf16 GEMM figure, the burst one only when no
-    sustained figure exists."""
-    if peaks.get("bf16_tflops_sustained"):
-        return peaks["bf16_tflops_sustained"], f"{peaks['source']} bf16 sustained (power-capped, back-to-back GEMM)"
-    return peaks["bf16_tflops"], f"{peaks['source']} bf16 burst"
+def check_device(P, when):
+    st, site = P.spk_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} at site {site} {when}")
 
 
-def exp2_peak_per_s():
-    """Exponentials per second the SMs can produce: the MUFU gives 16 ex2 per
-    clock per SM; the FMA pipe (128 lanes) spends 2 lane-ops per logit on the
-    scale and the sum and 7 per polynomial exponential, so the best split
-    (40 % polynomial) reaches 16 / 0.6 = 26.7 exponentials per clock per SM."""
-    return 148 * (16.0 / 0.6) * 1965e6
-
-
-# The files that define the scoring kernels and how they are launched.
-SCORING_SOURCES = ("api.cu", "common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh")
-
-
-def kernel_source_digest():
-    """sha256 over the scoring kernels' sources (SCORING_SOURCES); the DRAM
-    traffic captured with ncu is only reported while they are unchanged."""
-    import hashlib
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "prompt_compression_b200", "csrc")
-    for name in SCORING_SOURCES:
-        h.update(name.encode())
-        h.update(open(os.path.join(csrc, name), "rb").read())
-    return h.hexdigest()
-
-
-def captured_traffic(kernel, workload):
-    """dram__bytes_read.sum + dram__bytes_write.sum per launch from
-    profiles/traffic.json, or None when absent or captured from other sources."""
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    try:
-        rec = json.load(open(prof))
-    except (OSError, ValueError):
-        return None
-    if rec.get("source_sha256") != kernel_source_digest():
-        return None
-    return rec.get(kernel, {}).get(workload)
-
-
-def time_oracle(units_payload, cores):
-    """Run the oracle on the given units over `cores` spawned processes; returns seconds."""
-    import multiprocessing as mp
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(processes=cores) as pool:
-        pool.map(_oracle_unit_job, units_payload[:1])          # warm: import + build
-        t0 = time.perf_counter()
-        pool.map(_oracle_unit_job, units_payload, chunksize=1)
-        return time.perf_counter() - t0
-
-
+# ----------------------------------------------------------------- oracle timing (CPU baseline)
 def host_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -226,50 +226,135 @@ def host_cores():
         return os.cpu_count() or 1
 
 
-def cpu_sample_payload(cfg, seed, n_units):
-    payload = []
-    for u in range(n_units):
+def _oracle_job(job):
+    """One oracle sample (fp64, single thread).  The process draws its own
+    seeded inputs first (not timed), then runs the oracle:
+      ("speckv", cfg, seed, unit, heads): scores -> pool -> top-C + window ->
+          gather of K and V for one unit (the rows of its first `heads` query
+          heads, or all of them);
+      ("specpc", cfg, seed, b, layer, heads): SpecPC scores of one scored
+          layer of batch element b (its first `heads` query heads and their
+          KV heads, or all of them), then pool + top-K.
+    Returns the oracle's wall seconds in this single-threaded process."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    kind, cfg, seed = job[0], job[1], job[2]
+    if kind == "speckv":
+        u, heads = job[3], job[4]
         qb, kb, vb = W.speckv_unit_numpy(cfg, seed, u)
-        payload.append((qb, kb, vb, cfg.n_window, cfg.n_lookahead, cfg.c_max, cfg.pool))
-    return payload
+        if heads is not None:
+            qb = np.ascontiguousarray(qb[:heads])
+        t0 = time.perf_counter()
+        s, p, idx = oracle.speckv_select_unit(qb, kb, cfg.n_window, cfg.n_lookahead, cfg.c_max, cfg.pool)
+        oracle.gather_rows(kb, idx)
+        oracle.gather_rows(vb, idx)
+        return time.perf_counter() - t0
+    b, layer, heads = job[3], job[4], job[5]
+    qb, kb = W.specpc_layer_numpy(cfg, seed, b, layer)
+    if heads is not None:
+        qb = np.ascontiguousarray(qb[:heads])
+        kb = np.ascontiguousarray(kb[:max(1, heads // cfg.g)])
+    w = W.specpc_row_weights(cfg.n_rows).astype(np.float32).astype(np.float64)
+    t0 = time.perf_counter()
+    s = oracle.specpc_batch(qb[None], kb[None], w, 0, cfg.n_lookahead)
+    oracle.topk_with_tail(oracle.maxpool(s, cfg.pool), cfg.keep, 0)
+    return time.perf_counter() - t0
+
+
+def run_oracle_pool(jobs, cores):
+    """Run the jobs over `cores` spawned single-threaded processes (spawned,
+    so that none inherits a CUDA context); returns each job's oracle seconds."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(processes=cores) as pool:
+        pool.map(_oracle_job, jobs[:1])                     # warm: import + build
+        return pool.map(_oracle_job, jobs, chunksize=1)
+
+
+def cpu_baseline_speckv(cfg, seed, cores, full=False):
+    """The oracle on all host cores, one single-threaded process per core.
+    full: every unit of the workload; else one sample per core, each a unit
+    restricted to one query head's rows (1/g of the unit's work).  value =
+    the work timed / (the summed oracle seconds / cores)."""
+    if full:
+        secs = run_oracle_pool([("speckv", cfg, seed, u, None) for u in range(cfg.units)], cores)
+        value = cfg.kv_head_tokens / (sum(secs) / cores)
+        sample = (f"all {cfg.units} units of {cfg.name}, one process per core on {cores} cores, "
+                  f"{sum(secs):.0f} oracle CPU-s")
+    else:
+        secs = run_oracle_pool([("speckv", cfg, seed, u % 8, 1) for u in range(cores)], cores)
+        value = cores * cfg.n_in / cfg.g / (sum(secs) / cores)
+        sample = (f"{cores} samples, one per core, each one unit of {cfg.name} restricted to the rows of 1 "
+                  f"of its {cfg.g} query heads (1/{cfg.g} unit), {sum(secs):.0f} oracle CPU-s; the full step "
+                  f"has {cfg.units} units")
+    return {"value": value, "unit": "KV-head-tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+
+def cpu_baseline_specpc(cfg, seed, cores):
+    """The whole SpecPC workload on the host cores: every (batch element,
+    scored layer) as its own oracle call; the final mean over layers and max
+    over heads (n_in additions per layer) is not timed."""
+    jobs = [("specpc", cfg, seed, b, l, None) for b in range(cfg.batch) for l in range(cfg.layers_used)]
+    secs = run_oracle_pool(jobs, cores)
+    return {"value": cfg.kv_head_tokens / (sum(secs) / cores), "unit": "KV-head-tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"the whole workload: {len(jobs)} (batch, layer) oracle calls of {cfg.name} over {cores} "
+                      f"cores, {sum(secs):.0f} oracle CPU-s"}
+
+
+def cpu_baseline_cascade(cc, seed, cores):
+    """Sampled and extrapolated: step 1 timed on one query head (with its KV
+    head) of every scored layer of one batch element, step 2 on up to `cores`
+    units of the gathered target cache; the CPU-seconds are scaled to the full
+    job and spread over the host cores."""
+    d, t = cc.draft, cc.target
+    s1 = run_oracle_pool([("specpc", d, seed, 0, l, 1) for l in range(d.layers_used)], cores)
+    tg = W.SpecKVConfig("cascade_target_2k", batch=t.batch, layers=t.layers, hq=t.hq, hkv=t.hkv,
+                        head_dim=t.head_dim, n_in=d.keep, n_window=t.n_window, n_lookahead=t.n_lookahead,
+                        c_max=t.c_max, heavy_frac=t.heavy_frac)
+    n2 = min(cores, tg.units)
+    s2 = run_oracle_pool([("speckv", tg, seed, u, None) for u in range(n2)], cores)
+    full_cpu = sum(s1) * d.batch * d.hq + sum(s2) * tg.units / n2
+    tokens = t.batch * t.layers * t.hkv * cc.n_in_full
+    return {"value": tokens / (full_cpu / cores), "unit": "target KV-head-tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"extrapolated: step 1 timed on 1 of {d.hq} query heads of one batch element "
+                      f"({sum(s1):.0f} CPU-s, x {d.batch * d.hq}), step 2 on {n2} of {tg.units} units "
+                      f"({sum(s2):.0f} CPU-s); {full_cpu:.0f} CPU-s over {cores} cores"}
 
 
 def run_reference(args, cfg):
-    """--impl reference: the fp64 oracle on the host cores, same metric."""
+    """--impl reference: the fp64 oracle on the host cores, same metric and
+    workload; each step is one sample per core (a unit restricted to one
+    query head's rows), all in parallel, and takes as long as its slowest
+    sample; the whole run stays within a few minutes."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
     oracle.build()
-    cores = min(host_cores(), 16)
-    per_step = cores                     # one sample per process per step
-    # Each sample is one unit restricted to the rows of one query head of its
-    # GQA group (1/g of the unit's work; the oracle's cost is linear in rows),
-    # so that the whole --steps/--warmup run stays within a few minutes.
-    payload = [(qb[:1], kb, vb, nw, nl, c, pl)
-               for (qb, kb, vb, nw, nl, c, pl) in cpu_sample_payload(cfg, args.seed, min(per_step, 4))]
-    payload = (payload * per_step)[:per_step]
+    cores = host_cores()
+    jobs = [("speckv", cfg, args.seed, u % 8, 1) for u in range(cores)]
     import multiprocessing as mp
     ctx = mp.get_context("spawn")
     times = []
     with ctx.Pool(processes=cores) as pool:
-        pool.map(_oracle_unit_job, payload[:1])
+        pool.map(_oracle_job, jobs[:1])
         for s in range(args.warmup + args.steps):
-            t0 = time.perf_counter()
-            pool.map(_oracle_unit_job, payload, chunksize=1)
+            secs = pool.map(_oracle_job, jobs, chunksize=1)
             if s >= args.warmup:
-                times.append(time.perf_counter() - t0)
+                times.append(max(secs))
     step = sum(times) / len(times)
-    value = per_step * cfg.n_in / cfg.g / step
-    sample = (f"{per_step} samples per step, one per process, each = one unit of {cfg.name} with the "
-              f"rows of 1 of its {cfg.g} query heads (1/{cfg.g} unit of work); the full step has "
-              f"{cfg.units} units")
+    value = cores * cfg.n_in / cfg.g / step
+    sample = (f"{cores} samples per step, one per core, each = one unit of {cfg.name} with the rows of 1 of "
+              f"its {cfg.g} query heads (1/{cfg.g} unit of work); a step lasts as long as its slowest sample; "
+              f"the full step has {cfg.units} units")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "KV-head-tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "units_per_step": per_step, "n_in": cfg.n_in,
+        "config": {"workload": cfg.name, "units_per_step": cores, "n_in": cfg.n_in,
                    "c_max": cfg.c_max, "pool": cfg.pool},
         "cpu_baseline": {"value": value, "unit": "KV-head-tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -302,39 +387,21 @@ def whole_job_value(world: int, units_tokens: int, steps: int, ms_total_max: flo
     return world * units_tokens * steps / (ms_total_max * 1e-3)
 
 
-# ----------------------------------------------------------------- GPU arm
-def main():
-    args = parse()
-    cfg = config_of(args)
-    if args.impl == "reference":
-        if not isinstance(cfg, W.SpecKVConfig):
-            print(json.dumps({"impl": "reference", "unavailable":
-                              "the CPU reference arm times the SpecKV workloads only"}))
-            return
-        run_reference(args, cfg)
-        return
-    if isinstance(cfg, W.DecodeConfig):
-        run_decode(args, cfg)
-        return
-    if not isinstance(cfg, W.SpecKVConfig):
-        run_other(args, cfg)
-        return
+def kernel_roofline(name, ms, flops, peaks, traffic=None):
+    """Roofline object of a tensor-bound scoring kernel from its in-step time."""
+    peak, src = tensor_peak(peaks)
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic, "peak_source": src,
+            "sustained_peak": peaks.get("bf16_tflops_sustained"),
+            "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                  if peaks.get("bf16_tflops_sustained") else None)}
 
+
+# ----------------------------------------------------------------- SpecKV workloads
+def run_speckv(args, cfg, P, dev, world, rank, headline):
     import torch
     import torch.distributed as dist
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-
-    from prompt_compression_b200 import build
-    build.build_library()
-    import prompt_compression_b200 as P
     from prompt_compression_b200.pipeline import SpeckvBuffers
 
     seed = rank_seed(args.seed, rank)
@@ -343,131 +410,81 @@ def main():
     buf = SpeckvBuffers(q, k, v, cfg.n_window, cfg.c_max)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        P.speckv_compress(q, k, v, cfg.n_window, cfg.c_max, cfg.pool, buffers=buf, stream=stream)
-
     def barrier():
         if world > 1:
             dist.barrier()
 
-    def max_ranks(x: float) -> float:
-        return max_over_ranks(x, world, dev)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    st, site = P.spk_device_error()
-    if st != 0:
-        raise RuntimeError(f"device error {st} at site {site} during warm-up")
-
-    # ---- timed region: K steps, events on the launching stream
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        time.sleep(0.3)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-    barrier()
-    ms_total = max_ranks(e0.elapsed_time(e1))
+    launches = [
+        ("score_lse_pass", lambda: P.speckv_row_offsets(q, k, cfg.n_window, buf.ws_score, stream=stream)),
+        ("score_colsum_pass", lambda: P.speckv_colsum(q, k, cfg.n_window, buf.scores, buf.ws_score,
+                                                      stream=stream)),
+        ("topk_select", lambda: P.topk_select(buf.scores, cfg.c_max, cfg.n_window, buf.idx, cfg.pool, None,
+                                              buf.ws_topk, stream=stream)),
+        ("kv_compact", lambda: P.kv_compact(k, v, buf.idx, buf.k_out, buf.v_out, 1, stream=stream)),
+    ]
+    total, per, med, clocks = timed_steps(launches, args.steps, args.warmup, stream, barrier)
+    check_device(P, "in the timed steps")
+    ms_total = max_over_ranks(total, world, dev)
     ms_step = ms_total / args.steps
     value = whole_job_value(world, cfg.kv_head_tokens, args.steps, ms_total)
 
-    # ---- per-kernel timing: pass 1 alone (row LSE), then the whole score call
-    lse2 = torch.empty((cfg.units, cfg.g * cfg.rows), dtype=torch.float32, device=dev)
-
-    def timed(fn, n):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        fn()
-        torch.cuda.synchronize()
-        a.record(stream)
-        for _ in range(n):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / n
-
-    n_k = max(3, min(args.steps, 10))
-    ms_lse = timed(lambda: P.speckv_row_lse(q, k, cfg.n_window, lse2, stream=stream), n_k)
-    ms_score = timed(lambda: P.speckv_score(q, k, cfg.n_window, buf.scores, None, buf.ws_score,
-                                            stream=stream), n_k)
-    ms_topk = timed(lambda: P.topk_select(buf.scores, cfg.c_max, cfg.n_window, buf.idx, cfg.pool, None,
-                                          buf.ws_topk, stream=stream), n_k)
-    ms_compact = timed(lambda: P.kv_compact(k, v, buf.idx, buf.k_out, buf.v_out, 1, stream=stream), n_k)
-    ms_colsum = ms_score - ms_lse
-    st, site = P.spk_device_error()
-    if st != 0:
-        raise RuntimeError(f"device error {st} at site {site}")
-
     peaks = load_peaks()
     flops_pass = algorithmic_flops(cfg)
+    peak, _ = tensor_peak(peaks)
     kernels = {
-        "score_lse_pass": {"ms": ms_lse, "tflops": flops_pass / (ms_lse * 1e-3) / 1e12},
-        "score_colsum_pass": {"ms": ms_colsum, "tflops": flops_pass / (ms_colsum * 1e-3) / 1e12},
-        "topk_select": {"ms": ms_topk},
-        "kv_compact": {"ms": ms_compact,
-                       "gbs": cfg.units * 4 * cfg.keep * cfg.head_dim * 2 / (ms_compact * 1e-3) / 1e9},
+        "score_lse_pass": {"ms": per["score_lse_pass"],
+                           "tflops": flops_pass / (per["score_lse_pass"] * 1e-3) / 1e12},
+        "score_colsum_pass": {"ms": per["score_colsum_pass"],
+                              "tflops": flops_pass / (per["score_colsum_pass"] * 1e-3) / 1e12},
+        "topk_select": {"ms": per["topk_select"],
+                        "gbs": topk_bytes(cfg.units, cfg.n_pre, cfg.keep) / (per["topk_select"] * 1e-3) / 1e9},
+        "kv_compact": {"ms": per["kv_compact"],
+                       "gbs": cfg.units * 4 * cfg.keep * cfg.head_dim * 2 / (per["kv_compact"] * 1e-3) / 1e9},
     }
-    dom = "score_lse_pass" if ms_lse >= ms_colsum else "score_colsum_pass"
-    achieved = kernels[dom]["tflops"]
-    peak, peak_src = tensor_peak(peaks)
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": captured_traffic(dom, cfg.name),
-                "peak_source": peak_src,
-                "step_roofline_ms": max(2 * flops_pass / (peak * 1e12),
-                                        algorithmic_bytes(cfg) / (peaks["hbm_gbs"] * 1e9)) * 1e3}
+    for name in ("score_lse_pass", "score_colsum_pass"):
+        kernels[name]["frac"] = kernels[name]["tflops"] / peak
+    for name in ("topk_select", "kv_compact"):
+        kernels[name]["frac_hbm"] = kernels[name]["gbs"] / peaks["hbm_gbs"]
+    dom = max(("score_lse_pass", "score_colsum_pass"), key=lambda n: per[n])
+    roofline = kernel_roofline(dom, per[dom], flops_pass, peaks, captured_traffic(dom, cfg.name))
+    roofline["step_roofline_ms"] = max(2 * flops_pass / (peak * 1e12),
+                                       algorithmic_bytes(cfg) / (peaks["hbm_gbs"] * 1e9)) * 1e3
     roofline["step_frac"] = roofline["step_roofline_ms"] / ms_step
+    roofline["kernel_ms_sum"] = sum(per.values())
 
-    # ---- e2e through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_ranks, barrier)
+    if headline and not args.no_e2e:
+        e2e = run_e2e(args, cfg, P, q, k, v, dev, stream, world, lambda x: max_over_ranks(x, world, dev), barrier)
+    del inp, q, k, v, buf
+    torch.cuda.empty_cache()
 
-    # ---- CPU baseline (oracle), rank 0 at N = 1 only
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        cores = host_cores()
-        n_units = max(1, min(cores, 8))
-        payload = cpu_sample_payload(cfg, args.seed, n_units)
-        secs = time_oracle(payload, n_units)
-        cpu = {"value": n_units * cfg.n_in / secs, "unit": "KV-head-tokens/s", "cores": n_units,
-               "kind": "oracle",
-               "sample": f"{n_units} units of {cfg.name} (one per process, seeded host inputs), "
-                         f"{secs:.1f} s wall; the full step has {cfg.units} units"}
+        cpu = cpu_baseline_speckv(cfg, args.seed, host_cores(), full=cfg.n_in <= 16384)
 
-    launches = 4 * args.steps
-    line = {
-        "metric": METRIC, "value": value, "unit": "KV-head-tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+    return {
+        "metric": METRIC if headline else f"KV-head-tokens scored+selected+compacted/s ({cfg.name}, C_max {cfg.c_max})",
+        "value": value, "unit": "KV-head-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_step_median": med,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "units": cfg.units, "layers": cfg.layers, "hq": cfg.hq,
                    "hkv": cfg.hkv, "head_dim": cfg.head_dim, "n_in": cfg.n_in, "n_window": cfg.n_window,
                    "n_lookahead": cfg.n_lookahead, "c_max": cfg.c_max, "pool": cfg.pool,
-                   "l2": f"inputs larger than L2 (K, V {k.numel() * 2 / 1e9:.1f} GB each); no flush",
+                   "l2": f"inputs larger than L2 (K, V {cfg.units * cfg.n_in * cfg.head_dim * 2 / 1e9:.2f} GB "
+                         f"each); no flush",
                    "parallelism": f"units sharded, {world} rank(s), no collective"},
-        "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
-        "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu,
+        "roofline": roofline, "kernels": kernels, "gpu_launches": len(launches) * args.steps,
+        "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
     }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
 
 
-def run_other(args, cfg):
-    """SpecPC (scores + pool + top-K prompt tokens over a draft) and the
-    SpecKV-PC cascade (SpecPC on the draft, gather of the target cache, SpecKV
-    on the gathered cache), one GPU, one JSON line."""
+# ----------------------------------------------------------------- SpecPC and the cascade
+def run_specpc_like(args, cfg, P, dev):
+    """SpecPC (scores + pool + top-K prompt tokens over a draft) or the
+    SpecKV-PC cascade (SpecPC on the draft, gather of the target cache,
+    SpecKV on the gathered cache), one GPU."""
     import torch
-    from prompt_compression_b200 import build
-    build.build_library()
-    import prompt_compression_b200 as P
     from prompt_compression_b200.pipeline import SpeckvBuffers
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     peaks = load_peaks()
     cascade = isinstance(cfg, W.CascadeConfig)
@@ -479,8 +496,17 @@ def run_other(args, cfg):
     shape = P.binding.specpc_shape(dr["q"], dr["k"], d.l_skip, d.n_lookahead)
     ws_pc = torch.empty(max(P.specpc_workspace_size(shape), 256), dtype=torch.uint8, device=dev)
     ws_tk = torch.empty(max(P.topk_workspace_size(d.batch, d.n_in), 256), dtype=torch.uint8, device=dev)
-    flops = 2 * specpc_flops(d)
-    launches_per_step = 3
+    pc_flops = specpc_flops(d)
+    # the column pass adds a merge launch when it splits the segments into groups
+    offsets = -(-(d.units * (-(-d.g * d.n_rows // 128)) * 4096) // 256) * 256
+    merge = ws_pc.numel() > max(offsets, 256)
+    launches = [
+        ("specpc_lse_pass", lambda: P.specpc_row_offsets(dr["q"], dr["k"], w, ws_pc, d.l_skip, d.n_lookahead,
+                                                         stream=stream)),
+        ("specpc_colsum_pass", lambda: P.specpc_colsum(dr["q"], dr["k"], pc_scores, ws_pc, d.l_skip,
+                                                       d.n_lookahead, stream=stream)),
+        ("specpc_topk", lambda: P.topk_select(pc_scores, d.keep, 0, pc_idx, d.pool, None, ws_tk, stream=stream)),
+    ]
     if cascade:
         t = cfg.target
         tfull = W.SpecKVConfig("cascade_target_full", batch=t.batch, layers=t.layers, hq=t.hq, hkv=t.hkv,
@@ -492,74 +518,82 @@ def run_other(args, cfg):
         buf = SpeckvBuffers(tg["q"], kg, vg, t.n_window, t.c_max)
         tcfg = W.SpecKVConfig("g", batch=t.batch, layers=t.layers, hq=t.hq, hkv=t.hkv, head_dim=t.head_dim,
                               n_in=d.keep, n_window=t.n_window, n_lookahead=t.n_lookahead, c_max=t.c_max)
-        flops += 2 * algorithmic_flops(tcfg)
-        launches_per_step += 1 + 4
+        launches += [
+            ("cascade_gather", lambda: P.kv_compact(tg["k"], tg["v"], pc_idx, kg, vg, t.layers * t.hkv,
+                                                    stream=stream)),
+            ("target_lse_pass", lambda: P.speckv_row_offsets(tg["q"], kg, t.n_window, buf.ws_score, stream=stream)),
+            ("target_colsum_pass", lambda: P.speckv_colsum(tg["q"], kg, t.n_window, buf.scores, buf.ws_score,
+                                                           stream=stream)),
+            ("target_topk", lambda: P.topk_select(buf.scores, t.c_max, t.n_window, buf.idx, t.pool, None,
+                                                  buf.ws_topk, stream=stream)),
+            ("target_compact", lambda: P.kv_compact(kg, vg, buf.idx, buf.k_out, buf.v_out, 1, stream=stream)),
+        ]
         tokens = t.batch * t.layers * t.hkv * cfg.n_in_full
         metric = "target KV-head-tokens compressed/s (SpecPC 128K -> 2048 -> SpecKV 256 + 64)"
+        unit = "target KV-head-tokens/s"
     else:
         tokens = d.kv_head_tokens
         metric = "KV-head-tokens scored+selected/s (SpecPC draft)"
-
-    def step():
-        P.specpc_score(dr["q"], dr["k"], w, pc_scores, d.l_skip, d.n_lookahead, ws_pc, stream=stream)
-        P.topk_select(pc_scores, d.keep, 0, pc_idx, d.pool, None, ws_tk, stream=stream)
-        if cascade:
-            P.kv_compact(tg["k"], tg["v"], pc_idx, kg, vg, t.layers * t.hkv, stream=stream)
-            P.speckv_compress(tg["q"], kg, vg, t.n_window, t.c_max, t.pool, buffers=buf, stream=stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    st, site = P.spk_device_error()
-    if st != 0:
-        raise RuntimeError(f"device error {st} at site {site} during warm-up")
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clk:
-        time.sleep(0.3)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-    ms_step = e0.elapsed_time(e1) / args.steps
-    achieved = flops / (ms_step * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "whole step (scoring passes dominate)", "achieved": achieved,
-                "peak": tensor_peak(peaks)[0], "unit": "TFLOP/s", "frac": achieved / tensor_peak(peaks)[0],
-                "traffic": None, "peak_source": tensor_peak(peaks)[1]}
-    if not cascade:
-        # head_dim 64 halves the tensor work per logit, so the exponential
-        # stream (one exp2 per visible logit per pass) is the binding ceiling
-        exps = 2 * specpc_flops(d) / (2 * d.head_dim)
-        peak_exp = exp2_peak_per_s() / 1e9
-        ach_exp = exps / (ms_step * 1e-3) / 1e9
-        roofline = {"bound": "alu", "kernel": "whole step (scoring passes dominate)", "achieved": ach_exp,
-                    "peak": peak_exp, "unit": "Gexp2/s", "frac": ach_exp / peak_exp, "traffic": None,
-                    "peak_source": "derived: 148 SMs x 26.7 exp2/clk (MUFU 16/clk + FMA-pipe polynomial) x 1965 MHz",
-                    "tensor_frac": achieved / tensor_peak(peaks)[0]}
-    line = {
-        "metric": metric, "value": tokens / (ms_step * 1e-3), "unit": "KV-head-tokens/s", "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        unit = "KV-head-tokens/s"
+    total, per, med, clocks = timed_steps(launches, args.steps, args.warmup, stream)
+    check_device(P, "in the timed steps")
+    ms_step = total / args.steps
+    # each SpecPC pass evaluates one exp2 per visible logit: the exponential
+    # stream binds at head_dim 64 (the tensor work per logit is halved)
+    exps = pc_flops / (2 * d.head_dim)
+    kernels = {}
+    for name in ("specpc_lse_pass", "specpc_colsum_pass"):
+        kernels[name] = {"ms": per[name], "tflops": pc_flops / (per[name] * 1e-3) / 1e12,
+                         "gexp2_per_s": exps / (per[name] * 1e-3) / 1e9}
+    for name in per:
+        kernels.setdefault(name, {"ms": per[name]})
+    dom = max(("specpc_lse_pass", "specpc_colsum_pass"), key=lambda n: per[n])
+    peak_exp = exp2_peak_per_s() / 1e9
+    ach_exp = exps / (per[dom] * 1e-3) / 1e9
+    roofline = {"bound": "alu", "kernel": dom, "achieved": ach_exp, "peak": peak_exp, "unit": "Gexp2/s",
+                "frac": ach_exp / peak_exp, "traffic": None,
+                "peak_source": "derived: 148 SMs x 26.7 exp2/clk (MUFU 16/clk + FMA-pipe polynomial) x 1965 MHz",
+                "tensor_frac": kernels[dom]["tflops"] / tensor_peak(peaks)[0],
+                "kernel_ms_sum": sum(per.values())}
+    if cascade:
+        tf = algorithmic_flops(tcfg)
+        for name in ("target_lse_pass", "target_colsum_pass"):
+            kernels[name]["tflops"] = tf / (per[name] * 1e-3) / 1e12
+        kernels["cascade_gather"]["gbs"] = (2 * 2 * t.batch * t.layers * t.hkv * d.keep * t.head_dim * 2
+                                            / (per["cascade_gather"] * 1e-3) / 1e9)
+        roofline["step_roofline_ms"] = (2 * pc_flops / (exp2_peak_per_s() * 2 * d.head_dim) * 1e3
+                                        + 2 * tf / (tensor_peak(peaks)[0] * 1e12) * 1e3)
+        roofline["step_frac"] = roofline["step_roofline_ms"] / ms_step
+    else:
+        roofline["step_roofline_ms"] = 2 * exps / exp2_peak_per_s() * 1e3
+        roofline["step_frac"] = roofline["step_roofline_ms"] / ms_step
+    del dr
+    if cascade:
+        del tg, kg, vg, buf
+    torch.cuda.empty_cache()
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = cpu_baseline_cascade(cfg, args.seed, host_cores()) if cascade else \
+            cpu_baseline_specpc(cfg, args.seed, host_cores())
+    return {
+        "metric": metric, "value": tokens / (ms_step * 1e-3), "unit": unit, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "ms_per_step_median": med,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "l2": "inputs larger than L2; no flush"},
-        "roofline": roofline,
-        "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(), "e2e": None,
-        "cpu_baseline": None,
+        "roofline": roofline, "kernels": kernels,
+        "gpu_launches": (len(launches) + (1 if merge else 0)) * args.steps,
+        "clocks": clocks, "e2e": None, "cpu_baseline": cpu,
     }
-    print(json.dumps(line), flush=True)
 
 
-def run_decode(args, cfg):
+# ----------------------------------------------------------------- decode over the compressed cache
+def run_decode(args, cfg, P, dev):
     """One decode step over the compressed cache (C_max + window rows per KV
-    head) on every (layer, query head), one JSON line; the same step over the
-    full cache is timed for contrast.  Four copies of the compressed cache are
-    used in rotation so that consecutive launches read 4 x 84 MB, more than
-    the L2; the full cache (17 GB) is far larger than the L2."""
+    head) on every (layer, query head); the same step over the full cache is
+    timed for contrast.  Four copies of the compressed cache are used in
+    rotation so that consecutive launches read 4 x 84 MB, more than the L2;
+    the full cache (17 GB) is far larger than the L2."""
     import torch
-    from prompt_compression_b200 import build
-    build.build_library()
-    import prompt_compression_b200 as P
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     gen = torch.Generator(device=dev).manual_seed(args.seed)
     B_, L, hq, hkv, d = cfg.batch, cfg.layers, cfg.hq, cfg.hkv, cfg.head_dim
@@ -573,35 +607,25 @@ def run_decode(args, cfg):
     vcs = [rnd(B_, L, hkv, cfg.n_kv, d) for _ in range(copies)]
     out = torch.empty((B_, L, hq, d), dtype=torch.float32, device=dev)
     scale = d ** -0.5
-
-    def timed(fn, n):
-        for i in range(max(3, args.warmup)):
-            fn(i)
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for i in range(n):
-            fn(i)
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / n
-
-    steps = max(args.steps, 20) * 10
-    with ClockSampler(dev.index) as clk:
-        time.sleep(0.3)
-        ms = timed(lambda i: P.decode_attention(qs[i % copies], kcs[i % copies], vcs[i % copies], out, scale,
-                                                stream), steps)
-    st, site = P.spk_device_error()
-    if st != 0:
-        raise RuntimeError(f"device error {st} at site {site}")
+    reps = 10
+    launches = [(f"decode_{i}", (lambda i=i: P.decode_attention(qs[i % copies], kcs[i % copies], vcs[i % copies],
+                                                               out, scale, stream)))
+                for i in range(reps)]
+    total, per, med, clocks = timed_steps(launches, max(args.steps, 20), max(3, args.warmup), stream)
+    check_device(P, "in the timed steps")
+    steps = max(args.steps, 20) * reps
+    ms = total / steps
     del kcs, vcs
     kf, vf = rnd(B_, L, hkv, cfg.n_kv_full, d), rnd(B_, L, hkv, cfg.n_kv_full, d)
-    ms_full = timed(lambda i: P.decode_attention(qs[0], kf, vf, out, scale, stream), max(args.steps, 5))
+    tf, _, _, _ = timed_steps([("full", lambda: P.decode_attention(qs[0], kf, vf, out, scale, stream))],
+                              max(args.steps, 5), 3, stream)
+    ms_full = tf / max(args.steps, 5)
     del kf, vf
+    torch.cuda.empty_cache()
     peaks = load_peaks()
     nbytes = cfg.units * cfg.n_kv * d * 2 * 2 + B_ * L * hq * d * (2 + 4)
     gbs = nbytes / (ms * 1e-3) / 1e9
-    line = {
+    return {
         "metric": "decode over the compressed cache: query-head tokens/s", "value": B_ * L * hq / (ms * 1e-3),
         "unit": "query-head tokens/s", "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup),
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -613,23 +637,55 @@ def run_decode(args, cfg):
                      "peak_source": f"{peaks['source']} HBM copy"},
         "full_cache": {"n_kv": cfg.n_kv_full, "ms_per_step": ms_full,
                        "gbs": cfg.units * cfg.n_kv_full * d * 4 / (ms_full * 1e-3) / 1e9},
-        "gpu_launches": steps, "clocks": clk.summary(), "e2e": None, "cpu_baseline": None,
+        "gpu_launches": steps, "clocks": clocks, "e2e": None, "cpu_baseline": None,
     }
-    print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- traffic bookkeeping
+# The files that define the scoring kernels and how they are launched.
+SCORING_SOURCES = ("api.cu", "common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh")
+
+
+def kernel_source_digest():
+    """sha256 over the scoring kernels' sources (SCORING_SOURCES); the DRAM
+    traffic captured with ncu is only reported while they are unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "prompt_compression_b200", "csrc")
+    for name in SCORING_SOURCES:
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
+def captured_traffic(kernel, workload):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch from
+    profiles/traffic.json, or None when absent or captured from other sources."""
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(prof))
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != kernel_source_digest():
+        return None
+    return rec.get(kernel, {}).get(workload)
+
+
+# ----------------------------------------------------------------- e2e
 def run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_over_ranks, barrier):
     """Same metric end to end from pinned host memory, through the public API.
 
     Per step, the (batch, layer) pairs are taken in `--e2e-chunks` groups.  Q
     and K of a group are copied to the device on a copy stream; the group is
-    scored, selected and compacted on the compute stream as soon as its copy
-    has landed (the next group's copy overlaps that work); the compacted K is
-    gathered from the device copy of K, the compacted V straight from the
-    pinned host V (only the selected rows cross the host link); the indices
-    and the compacted K/V go back to pinned host memory on a third stream.
-    The timed region runs from before the first copy to the end of the last
-    copy back.  If the host V cannot be read in place, it is copied like K."""
+    scored, selected and compacted (speckv_compress) on the compute stream as
+    soon as its copy has landed (the next group's copy overlaps that work);
+    the compacted K is gathered from the device copy of K, the compacted V
+    straight from the pinned host V (only the selected rows cross the host
+    link); the indices and the compacted K/V go back to pinned host memory on
+    a third stream.  Each timed step runs from before its first copy to the
+    end of its last copy back (events on the compute stream); the line
+    reports the mean and the median step.  If the host V cannot be read in
+    place, it is copied like K."""
     import torch
     from prompt_compression_b200.pipeline import SpeckvBuffers
     need = (q.numel() + k.numel() + v.numel()) * 2
@@ -692,20 +748,73 @@ def run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_over_ranks, barrier):
     step()
     torch.cuda.synchronize()
     barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(args.e2e_steps):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.e2e_steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.e2e_steps):
         step()
-    b.record(stream)
+        ev[i + 1].record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(a.elapsed_time(b)) / args.e2e_steps
+    ms = max_over_ranks(ev[0].elapsed_time(ev[-1])) / args.e2e_steps
+    per_step = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(args.e2e_steps))
     keep_rows = sum(g[5].idx.numel() for g in groups)
     h2d = (q.numel() + k.numel()) * 2 + (keep_rows * cfg.head_dim * 2 if v_in_place else v.numel() * 2)
     d2h = sum(g[6][0].numel() * 4 + (g[6][1].numel() + g[6][2].numel()) * 2 for g in groups)
     return {"value": world * cfg.kv_head_tokens / (ms * 1e-3), "unit": "KV-head-tokens/s",
-            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms, "ms_per_step_median": per_step[len(per_step) // 2],
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": args.e2e_steps, "groups": n_chunks,
             "v": "selected rows read in place from pinned host memory" if v_in_place else "copied"}
+
+
+# ----------------------------------------------------------------- main
+def main(argv=None):
+    args = parse(argv)
+    cfg = config_of(args.config, args.cmax)
+    if args.impl == "reference":
+        if not isinstance(cfg, W.SpecKVConfig):
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the CPU reference arm times the SpecKV workloads only"}))
+            return
+        run_reference(args, cfg)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from prompt_compression_b200 import build
+    build.build_library()
+    import prompt_compression_b200 as P
+
+    names = SUITE if args.suite else (args.config + (f"@{args.cmax}" if args.cmax else ""),)
+    lines = []
+    for name in names:
+        c = config_of(name)
+        headline = (c == W.QWEN32B_64K)
+        if isinstance(c, W.SpecKVConfig):
+            line = run_speckv(args, c, P, dev, world, rank, headline)
+        elif world > 1:
+            continue                         # the other workloads are single-GPU lines
+        elif isinstance(c, W.DecodeConfig):
+            line = run_decode(args, c, P, dev)
+        else:
+            line = run_specpc_like(args, c, P, dev)
+        lines.append((headline, line))
+        if rank == 0 and args.suite:
+            print(json.dumps(line), flush=True)
+        torch.cuda.empty_cache()
+    if rank == 0 and not args.suite:
+        print(json.dumps(lines[-1][1]), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
 
 
 if __name__ == "__main__":

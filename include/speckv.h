@@ -90,6 +90,21 @@ spk_status speckv_score(const spk_speckv_shape* shape, const void* q_bf16, const
                         float* scores, float* window_mass, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* The two passes of speckv_score as separate calls, for callers that time
+ * or schedule them apart; speckv_score is exactly speckv_row_offsets
+ * followed by speckv_colsum on the same stream.
+ *   speckv_row_offsets: pass 1 -- every query row's log-sum-exp, stored in the
+ *     workspace as the row offsets pass 2 adds to its logits;
+ *   speckv_colsum: pass 2 -- the scores (and window mass) from a workspace that
+ *     speckv_row_offsets filled for the same shape, q and k (ordered before
+ *     this call; the workspace is only read).
+ * Same shapes, layouts, workspace size and rules as speckv_score. */
+spk_status speckv_row_offsets(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+spk_status speckv_colsum(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16, float* scores,
+                         float* window_mass, const void* workspace, size_t workspace_bytes, void* stream);
+
 /* Pass 1 alone (diagnostic): the log2-domain log-sum-exp of every query row,
  * lse2[u][qh_local * R + i] = log2 sum_{visible j} 2^(scale*log2(e) * q.k_j),
  * fp32 [units][g * R].  Same shapes and rules as speckv_score. */
@@ -109,6 +124,9 @@ spk_status speckv_row_lse(const spk_speckv_shape* shape, const void* q_bf16, con
  *   - Every GPU that loads the library holds the 16 MiB until process exit.
  *   - The first call on a device looks up the array's address on that device
  *     (cudaGetSymbolAddress) and caches it: make it before any stream capture.
+ *     A cudaDeviceReset unloads the library's device image, so the cached
+ *     address is stale afterwards: do not call this entry point again in a
+ *     process that has reset the device.
  *   - All calls share the array, which keeps the last call's contents (every
  *     entry read is first rewritten by the same call, so nothing needs
  *     clearing); calls whose kernels overlap on the GPU race on it. */
@@ -127,10 +145,11 @@ spk_status speckv_score_static_ws(const spk_speckv_shape* shape, const void* q_b
  *
  *   q            bf16 [batch][layers][hq][W][head_dim]   (layers < l_skip are not read)
  *   k            bf16 [batch][layers][hkv][n_in][head_dim]
- *   row_weights  fp32 [W], device, oldest row first, w_i >= 0, sum > 0
+ *   row_weights  fp32 [W], device, oldest row first, w_i >= 0, sum > 0; a row
+ *                of weight 0 contributes nothing (its attention is not read)
  *   scores       fp32 [batch][n_in]
  *
- * Supported: head_dim == 64; hq % hkv == 0; hq <= 32; (hq/hkv) * W <= 2048;
+ * Supported: head_dim in {64, 128}; hq % hkv == 0; hq <= 32; (hq/hkv) * W <= 2048;
  * 0 <= l_skip < layers; 1 <= W <= n_in + n_lookahead - 1; n_lookahead >= 1.
  * ------------------------------------------------------------------------ */
 typedef struct {
@@ -139,20 +158,38 @@ typedef struct {
   float scale;
 } spk_specpc_shape;
 
-/* Workspace: units * ceil((hq/hkv) * W / 128) * 4096 bytes (rounded up to
- * 256), units = batch * (layers - l_skip) * hkv; 16-byte aligned. */
+/* Workspace: the row offsets, units * ceil((hq/hkv) * W / 128) * 4096 bytes
+ * (rounded up to 256), units = batch * (layers - l_skip) * hkv; when the
+ * column pass would leave SMs of the current device idle (few 256-key blocks,
+ * e.g. batch 1 at 32K), it splits each block's (KV head, layer) segments into
+ * G groups (G <= 16, chosen from the device's SM count) and adds
+ * batch * ceil(n_in / 256) * G * hq * 1 KB of per-head partial sums, which a
+ * merge kernel adds in a fixed order (results stay bitwise reproducible on a
+ * given device).  Query the size with the device current; 16-byte aligned. */
 size_t specpc_workspace_size(const spk_specpc_shape* shape);
 
 spk_status specpc_score(const spk_specpc_shape* shape, const void* q_bf16, const void* k_bf16,
                         const float* row_weights, float* scores, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* The two passes of specpc_score as separate calls (specpc_score is exactly
+ * specpc_row_offsets followed by specpc_colsum on the same stream): the row
+ * offsets with the row weights folded in, then the scores from them. */
+spk_status specpc_row_offsets(const spk_specpc_shape* shape, const void* q_bf16, const void* k_bf16,
+                              const float* row_weights, void* workspace, size_t workspace_bytes, void* stream);
+
+spk_status specpc_colsum(const spk_specpc_shape* shape, const void* q_bf16, const void* k_bf16, float* scores,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Pooling + top-k selection (section 关键设计: keep the top-C_max KV pairs plus
  * the window; section 损失函数 / 训练策略: local pooling keeps token runs)
  *
- * For each of `units` rows of n_cand candidate scores:
- *   pooled[j] = max scores[t] over t in [j - r, j + r] ∩ [0, n_cand), r = pool_kernel / 2
+ * For each of `units` rows of n_cand candidate scores, r = pool_kernel / 2 and
+ * W_j = [j - r, j + r] ∩ [0, n_cand) (the window clipped at the row's ends):
+ *   pooled[j] = max of scores over W_j                 (SPK_POOL_MAX)
+ *             = (sum of scores over W_j) / |W_j|       (SPK_POOL_AVG; fp32, summed
+ *               in index order, one correctly rounded division)
  *   selected  = the min(k, n_cand) largest pooled values; equal values are
  *               taken lowest index first
  *   idx[u]    = selected indices in ascending order, then the tail
@@ -162,12 +199,28 @@ spk_status specpc_score(const spk_specpc_shape* shape, const void* q_bf16, const
  *   idx     int32 [units][min(k, n_cand) + n_tail]
  *   pooled  fp32 [units][n_cand] or NULL
  *
- * Supported: pool_kernel odd >= 1; k >= 0; n_tail >= 0; n_cand >= 0.
+ * The pages say "local pooling" without its kind; the workloads use max
+ * pooling, which is what topk_select does.  topk_select_pool takes the mode.
+ * The workspace is used only when k > 2048 or more than 2048 pooled values
+ * fall into the 12-bit key bin of the k-th largest (long runs of equal
+ * values); it must always be given.
+ *
+ * Supported: pool_kernel odd >= 1; k >= 0; n_tail >= 0; n_cand >= 0;
+ * pool_mode SPK_POOL_MAX or SPK_POOL_AVG.
  * ------------------------------------------------------------------------ */
+typedef enum {
+  SPK_POOL_MAX = 0,
+  SPK_POOL_AVG = 1
+} spk_pool_mode;
+
 size_t topk_workspace_size(int units, int n_cand);
 
 spk_status topk_select(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail,
                        int32_t* idx, float* pooled, void* workspace, size_t workspace_bytes, void* stream);
+
+spk_status topk_select_pool(const float* scores, int units, int n_cand, int pool_mode, int pool_kernel, int k,
+                            int n_tail, int32_t* idx, float* pooled, void* workspace, size_t workspace_bytes,
+                            void* stream);
 
 /* ------------------------------------------------------------------------
  * KV compaction (section 关键设计, SpecKV: the dropped cache keeps only the

@@ -1,9 +1,12 @@
 """ctypes binding of include/speckv.h: argument marshalling only.
 
-Each function takes torch tensors that already live on the GPU, checks dtype,
-device and contiguity, and passes raw pointers, sizes and the current CUDA
-stream to the C entry point of the same name.  Output tensors are the
-caller's; a workspace is allocated with torch only when none is given.
+Each function takes torch tensors that already live on the GPU, checks their
+sizes, dtype, device and contiguity, and passes raw pointers, sizes and the
+CUDA stream to the C entry point of the same name.  The C ABI cannot see how
+large a buffer is, so every output's element count is checked here against
+the shape the entry point will write (ValueError on a mismatch) before the
+call.  Output tensors are the caller's; a workspace is allocated with torch
+only when none is given, and then on the stream the kernels run on.
 """
 from __future__ import annotations
 
@@ -60,10 +63,15 @@ def load_library():
         "speckv_workspace_size": (sz, [sk]),
         "speckv_score": (I, [sk, vp, vp, vp, vp, vp, sz, vp]),
         "speckv_row_lse": (I, [sk, vp, vp, vp, vp]),
+        "speckv_row_offsets": (I, [sk, vp, vp, vp, sz, vp]),
+        "speckv_colsum": (I, [sk, vp, vp, vp, vp, vp, sz, vp]),
         "specpc_workspace_size": (sz, [sp]),
         "specpc_score": (I, [sp, vp, vp, vp, vp, vp, sz, vp]),
+        "specpc_row_offsets": (I, [sp, vp, vp, vp, vp, sz, vp]),
+        "specpc_colsum": (I, [sp, vp, vp, vp, vp, sz, vp]),
         "topk_workspace_size": (sz, [I, I]),
         "topk_select": (I, [vp, I, I, I, I, I, vp, vp, vp, sz, vp]),
+        "topk_select_pool": (I, [vp, I, I, I, I, I, I, vp, vp, vp, sz, vp]),
         "kv_compact": (I, [vp, vp, I, I, I, I, vp, I, I, vp, vp, vp]),
         "spk_last_error": (ctypes.c_char_p, []),
         "spk_device_error": (I, [ctypes.POINTER(I), ctypes.POINTER(I), I]),
@@ -86,12 +94,34 @@ def _check(status: int):
         raise SpeckvError(status, msg)
 
 
+SPK_POOL_MAX, SPK_POOL_AVG = 0, 1
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+def _stream_object(stream, device):
+    """The torch stream the kernels will run on (a raw handle is wrapped)."""
+    if stream is None:
+        return torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return stream
+    return torch.cuda.ExternalStream(int(stream), device=device)
+
+
+def _numel(t: Optional[torch.Tensor], name: str, expected: int, required: bool = True):
+    """An output (or input) must hold exactly the elements the kernel touches."""
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return
+    if t.numel() != expected:
+        raise ValueError(f"{name} has {t.numel()} elements, the call needs {expected}")
 
 
 def _dev(t: Optional[torch.Tensor], name: str, dtype=None) -> Optional[int]:
@@ -124,10 +154,15 @@ def _src(t: Optional[torch.Tensor], name: str) -> Optional[int]:
     return mapped_host_pointer(t)
 
 
-def _workspace(ws: Optional[torch.Tensor], nbytes: int, device) -> torch.Tensor:
-    if ws is None:
+def _workspace(ws: Optional[torch.Tensor], nbytes: int, device, stream=None) -> torch.Tensor:
+    """The caller's workspace, or a temporary one.  A temporary is allocated
+    on the stream the kernels are enqueued on: the caching allocator then
+    hands its memory to later allocations of that stream only, which run
+    after the kernels, although the tensor is released when the call returns."""
+    if ws is not None:
+        return ws
+    with torch.cuda.stream(_stream_object(stream, device)):
         return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
-    return ws
 
 
 # --------------------------------------------------------------------- SpecKV
@@ -150,8 +185,11 @@ def speckv_score(q, k, n_window: int, scores, window_mass=None, workspace=None, 
     """scores[u][j] (and window_mass[u][j]) for every unit u = (b, layer, KV head)."""
     lib = load_library()
     shape = speckv_shape(q, k, n_window, scale)
+    units = shape.batch * shape.layers * shape.hkv
+    _numel(scores, "scores", units * (shape.n_in - n_window), required=shape.n_in > n_window)
+    _numel(window_mass, "window_mass", units * n_window, required=False)
     need = speckv_workspace_size(shape)
-    ws = _workspace(workspace, need, q.device)
+    ws = _workspace(workspace, need, q.device, stream)
     _check(lib.speckv_score(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
                             _dev(scores, "scores", torch.float32),
                             _dev(window_mass, "window_mass", torch.float32),
@@ -159,9 +197,38 @@ def speckv_score(q, k, n_window: int, scores, window_mass=None, workspace=None, 
     return scores
 
 
+def speckv_row_offsets(q, k, n_window: int, workspace, scale: float = 1.0, stream=None):
+    """Pass 1 of speckv_score: the row offsets, written into `workspace`."""
+    lib = load_library()
+    shape = speckv_shape(q, k, n_window, scale)
+    if workspace is None:
+        raise ValueError("workspace is required (speckv_workspace_size bytes)")
+    _check(lib.speckv_row_offsets(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
+                                  _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)))
+    return workspace
+
+
+def speckv_colsum(q, k, n_window: int, scores, workspace, window_mass=None, scale: float = 1.0, stream=None):
+    """Pass 2 of speckv_score, from a workspace speckv_row_offsets filled."""
+    lib = load_library()
+    shape = speckv_shape(q, k, n_window, scale)
+    units = shape.batch * shape.layers * shape.hkv
+    _numel(scores, "scores", units * (shape.n_in - n_window), required=shape.n_in > n_window)
+    _numel(window_mass, "window_mass", units * n_window, required=False)
+    if workspace is None:
+        raise ValueError("workspace is required (the one speckv_row_offsets filled)")
+    _check(lib.speckv_colsum(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
+                             _dev(scores, "scores", torch.float32), _dev(window_mass, "window_mass", torch.float32),
+                             _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                             _stream(stream)))
+    return scores
+
+
 def speckv_row_lse(q, k, n_window: int, lse2, scale: float = 1.0, stream=None):
     lib = load_library()
     shape = speckv_shape(q, k, n_window, scale)
+    _numel(lse2, "lse2", shape.batch * shape.layers * shape.hq * (shape.n_window + shape.n_lookahead))
     _check(lib.speckv_row_lse(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
                               _dev(lse2, "lse2", torch.float32), _stream(stream)))
     return lse2
@@ -172,7 +239,9 @@ def specpc_shape(q, k, l_skip: int, n_lookahead: int, scale: float = 1.0) -> Spe
     if q.dim() != 5 or k.dim() != 5:
         raise ValueError("q is [B, L, Hq, W, d] and k is [B, L, Hkv, n_in, d]")
     B, L, hq, W, d = q.shape
-    _, _, hkv, n_in, _ = k.shape
+    Bk, Lk, hkv, n_in, dk = k.shape
+    if (B, L, d) != (Bk, Lk, dk):
+        raise ValueError("q and k disagree on batch, layers or head_dim")
     return SpecpcShape(B, L, l_skip, hq, hkv, d, n_in, W, n_lookahead, float(scale))
 
 
@@ -184,11 +253,40 @@ def specpc_score(q, k, row_weights, scores, l_skip: int, n_lookahead: int = 1, w
                  scale: float = 1.0, stream=None):
     lib = load_library()
     shape = specpc_shape(q, k, l_skip, n_lookahead, scale)
-    ws = _workspace(workspace, specpc_workspace_size(shape), q.device)
+    _numel(row_weights, "row_weights", shape.n_rows)
+    _numel(scores, "scores", shape.batch * shape.n_in)
+    ws = _workspace(workspace, specpc_workspace_size(shape), q.device, stream)
     _check(lib.specpc_score(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
                             _dev(row_weights, "row_weights", torch.float32),
                             _dev(scores, "scores", torch.float32), _dev(ws, "workspace"),
                             ws.numel() * ws.element_size(), _stream(stream)))
+    return scores
+
+
+def specpc_row_offsets(q, k, row_weights, workspace, l_skip: int, n_lookahead: int = 1, scale: float = 1.0,
+                       stream=None):
+    """Pass 1 of specpc_score into `workspace`."""
+    lib = load_library()
+    shape = specpc_shape(q, k, l_skip, n_lookahead, scale)
+    _numel(row_weights, "row_weights", shape.n_rows)
+    if workspace is None:
+        raise ValueError("workspace is required (specpc_workspace_size bytes)")
+    _check(lib.specpc_row_offsets(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
+                                  _dev(row_weights, "row_weights", torch.float32), _dev(workspace, "workspace"),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+    return workspace
+
+
+def specpc_colsum(q, k, scores, workspace, l_skip: int, n_lookahead: int = 1, scale: float = 1.0, stream=None):
+    """Pass 2 of specpc_score from a workspace specpc_row_offsets filled."""
+    lib = load_library()
+    shape = specpc_shape(q, k, l_skip, n_lookahead, scale)
+    _numel(scores, "scores", shape.batch * shape.n_in)
+    if workspace is None:
+        raise ValueError("workspace is required (the one specpc_row_offsets filled)")
+    _check(lib.specpc_colsum(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
+                             _dev(scores, "scores", torch.float32), _dev(workspace, "workspace"),
+                             workspace.numel() * workspace.element_size(), _stream(stream)))
     return scores
 
 
@@ -198,14 +296,25 @@ def topk_workspace_size(units: int, n_cand: int) -> int:
 
 
 def topk_select(scores, k: int, n_tail: int, idx, pool_kernel: int = 7, pooled=None, workspace=None,
-                stream=None):
-    """scores [units, n_cand] fp32 -> idx [units, min(k, n_cand) + n_tail] int32."""
+                stream=None, pool_mode: int = SPK_POOL_MAX):
+    """scores [units, n_cand] fp32 -> idx [units, min(k, n_cand) + n_tail] int32.
+    pool_mode SPK_POOL_MAX (topk_select) or SPK_POOL_AVG (topk_select_pool)."""
     lib = load_library()
+    if scores.dim() != 2:
+        raise ValueError("scores is [units, n_cand]")
     units, n_cand = scores.shape
-    ws = _workspace(workspace, topk_workspace_size(units, n_cand), scores.device)
-    _check(lib.topk_select(_dev(scores, "scores", torch.float32), units, n_cand, pool_kernel, k, n_tail,
-                           _dev(idx, "idx", torch.int32), _dev(pooled, "pooled", torch.float32),
-                           _dev(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)))
+    if k < 0 or n_tail < 0:
+        raise ValueError("k and n_tail must be >= 0")
+    _numel(idx, "idx", units * (min(k, n_cand) + n_tail), required=units * (min(k, n_cand) + n_tail) > 0)
+    _numel(pooled, "pooled", units * n_cand, required=False)
+    ws = _workspace(workspace, topk_workspace_size(units, n_cand), scores.device, stream)
+    args = (_dev(scores, "scores", torch.float32), units, n_cand)
+    tail = (pool_kernel, k, n_tail, _dev(idx, "idx", torch.int32), _dev(pooled, "pooled", torch.float32),
+            _dev(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream))
+    if pool_mode == SPK_POOL_MAX:
+        _check(lib.topk_select(*args, *tail))
+    else:
+        _check(lib.topk_select_pool(*args, int(pool_mode), *tail))
     return idx
 
 
@@ -213,9 +322,25 @@ def kv_compact(k, v, idx, k_out, v_out, units_per_idx: int = 1, stream=None):
     """k, v [units, n_src, d] (any 2-byte or 4-byte dtype); idx [units/units_per_idx, n_idx].
     k and v may be CUDA tensors or pinned host tensors (gathered in place)."""
     lib = load_library()
+    if k.dim() < 2:
+        raise ValueError("k is [..., n_src, head_dim]")
     n_src, d = k.shape[-2], k.shape[-1]
     units = k.numel() // (n_src * d) if n_src * d else 0
+    if units_per_idx < 1 or units % units_per_idx:
+        raise ValueError(f"units ({units}) must be a multiple of units_per_idx ({units_per_idx})")
     n_idx = idx.shape[-1]
+    _numel(idx, "idx", units // units_per_idx * n_idx)
+    _numel(k_out, "k_out", units * n_idx * d)
+    if k_out.element_size() != k.element_size():
+        raise ValueError("k_out must have k's element size")
+    if (v is None) != (v_out is None):
+        raise ValueError("v and v_out are given together or not at all")
+    if v is not None:
+        if tuple(v.shape) != tuple(k.shape) or v.element_size() != k.element_size():
+            raise ValueError("v must have k's shape and element size")
+        _numel(v_out, "v_out", units * n_idx * d)
+        if v_out.element_size() != k.element_size():
+            raise ValueError("v_out must have k's element size")
     _check(lib.kv_compact(_src(k, "k"), _src(v, "v"), units, n_src, d, k.element_size(),
                           _dev(idx, "idx", torch.int32), n_idx, units_per_idx, _dev(k_out, "k_out"),
                           _dev(v_out, "v_out"), _stream(stream)))
@@ -226,10 +351,15 @@ def decode_attention(q, k, v, out=None, scale: float = 1.0, stream=None):
     """Decode attention over a compacted cache: q [B, L, Hq, d], k/v [B, L, Hkv, n_kv, d]
     (bf16, CUDA) -> out fp32 [B, L, Hq, d]."""
     lib = load_library()
+    if q.dim() != 4 or k.dim() != 5 or v.dim() != 5:
+        raise ValueError("q is [B, L, Hq, d]; k and v are [B, L, Hkv, n_kv, d]")
     Bsz, L, hq, d = q.shape
     hkv, n_kv = k.shape[2], k.shape[3]
+    if tuple(k.shape) != (Bsz, L, hkv, n_kv, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, L, Hkv, n_kv, d] with q's B, L and d")
     if out is None:
         out = torch.empty((Bsz, L, hq, d), dtype=torch.float32, device=q.device)
+    _numel(out, "out", Bsz * L * hq * d)
     _check(lib.decode_attention(Bsz, L, hq, hkv, d, n_kv, float(scale), _dev(q, "q", torch.bfloat16),
                                 _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
                                 _dev(out, "out", torch.float32), _stream(stream)))

@@ -188,8 +188,30 @@ spk_status speckv_row_lse(const spk_speckv_shape* s, const void* q, const void* 
   return st == SPK_OK ? ok() : st;
 }
 
-spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k, float* scores,
-                        float* window_mass, void* ws, size_t ws_bytes, void* stream) {
+// Pass 1 into the workspace: every query row's offset -lse2/c2 as the
+// operand blocks of pass 2's extra UMMA K-step.
+spk_status speckv_row_offsets(const spk_speckv_shape* s, const void* q, const void* k, void* ws, size_t ws_bytes,
+                              void* stream) {
+  SpeckvGeom g;
+  spk_status st = check_speckv(s, g);
+  if (st != SPK_OK) return st;
+  const size_t need = speckv_workspace_size(s);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
+  CUtensorMap qmap, kmap;
+  if ((st = speckv_maps(s, q, k, g, &qmap, &kmap)) != SPK_OK) return st;
+  ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
+                              s->layers, 0);
+  p.off_blocks = static_cast<uint8_t*>(ws);
+  p.off_tiles = static_cast<int>(row_tiles(g.rows));
+  st = run_lse(p, qmap, kmap, s->head_dim, static_cast<cudaStream_t>(stream));
+  return st == SPK_OK ? ok() : st;
+}
+
+// Pass 2 from a workspace that speckv_row_offsets filled for the same shape, q and k.
+spk_status speckv_colsum(const spk_speckv_shape* s, const void* q, const void* k, float* scores, float* window_mass,
+                         const void* ws, size_t ws_bytes, void* stream) {
   SpeckvGeom g;
   spk_status st = check_speckv(s, g);
   if (st != SPK_OK) return st;
@@ -202,12 +224,10 @@ spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k,
   if (n_cols == 0) return ok();
   CUtensorMap qmap, kmap;
   if ((st = speckv_maps(s, q, k, g, &qmap, &kmap)) != SPK_OK) return st;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
   ScoreParams p = base_params(s->head_dim, s->n_in, g, s->n_in - s->n_window + 1, s->scale, s->hkv, s->layers,
                               s->layers, 0);
-  p.off_blocks = static_cast<uint8_t*>(ws);
+  p.off_blocks = static_cast<uint8_t*>(const_cast<void*>(ws));
   p.off_tiles = static_cast<int>(row_tiles(g.rows));
-  if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
   p.n_pre = static_cast<int>(g.n_pre);
   p.n_cols = n_cols;
   p.out0 = scores;
@@ -215,9 +235,24 @@ spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k,
   p.n_blocks = (n_cols + 255) / 256;
   p.n_items = p.n_units * p.n_blocks;
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
-  cudaError_t e = launch_score(MODE_COLSUM, s->head_dim, kmap, qmap, p, grid, cs);
+  cudaError_t e = launch_score(MODE_COLSUM, s->head_dim, kmap, qmap, p, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
   return ok();
+}
+
+spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k, float* scores,
+                        float* window_mass, void* ws, size_t ws_bytes, void* stream) {
+  SpeckvGeom g;
+  spk_status st = check_speckv(s, g);
+  if (st != SPK_OK) return st;
+  if (g.n_pre > 0 && scores == nullptr) return fail(SPK_ERR_ARG, "scores must be non-NULL when n_window < n_in");
+  const size_t need = speckv_workspace_size(s);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
+  if ((window_mass ? s->n_in : g.n_pre) == 0) return ok();
+  if ((st = speckv_row_offsets(s, q, k, ws, ws_bytes, stream)) != SPK_OK) return st;
+  return speckv_colsum(s, q, k, scores, window_mass, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ SpecPC
@@ -231,7 +266,8 @@ static spk_status check_specpc(const spk_specpc_shape* s, SpeckvGeom& g) {
   if (static_cast<long long>(s->n_rows) > static_cast<long long>(s->n_in) + s->n_lookahead - 1)
     return fail(SPK_ERR_ARG, "n_rows must be <= n_in + n_lookahead - 1");
   if (!(s->scale > 0.f) || !std::isfinite(s->scale)) return fail(SPK_ERR_ARG, "scale must be finite and > 0");
-  if (s->head_dim != 64) return fail(SPK_ERR_UNSUPPORTED, "SpecPC supports head_dim 64 (got %d)", s->head_dim);
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(SPK_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", s->head_dim);
   g.g = s->hq / s->hkv;
   if (s->hq > kHeadsMax) return fail(SPK_ERR_UNSUPPORTED, "hq = %d exceeds %d", s->hq, kHeadsMax);
   g.R = s->n_rows;
@@ -245,10 +281,109 @@ static spk_status check_specpc(const spk_specpc_shape* s, SpeckvGeom& g) {
   return SPK_OK;
 }
 
+// SpecPC column pass: items are (batch element, 256-key block) pairs; when
+// they would leave SMs idle, each block's (KV head, layer) segments are split
+// into `groups` contiguous groups, one item each, whose per-head partial sums
+// a merge kernel adds in a fixed order.  groups is the smallest count, up to
+// 16 and to the number of segments, that fills the grid's waves to >= 95 %
+// (else the best fill found).
+static int specpc_groups(long long items, int nseg, int sms) {
+  auto fill = [&](int gcount) {
+    const long long n = items * gcount;
+    const long long waves = (n + sms - 1) / sms;
+    return static_cast<double>(n) / static_cast<double>(waves * sms);
+  };
+  int best = 1;
+  double best_fill = fill(1);
+  for (int gcount = 1; gcount <= 16 && gcount <= nseg; ++gcount) {
+    const double f = fill(gcount);
+    if (f >= 0.95) return gcount;
+    if (f > best_fill + 1e-9) { best = gcount; best_fill = f; }
+  }
+  return best;
+}
+
+struct SpecpcPlan {
+  int n_blocks, groups;
+  size_t off_bytes, part_bytes;
+};
+
+static SpecpcPlan specpc_plan(const spk_specpc_shape* s, const SpeckvGeom& g) {
+  SpecpcPlan pl;
+  pl.n_blocks = (s->n_in + 255) / 256;
+  pl.groups = specpc_groups(static_cast<long long>(s->batch) * pl.n_blocks, s->hkv * (s->layers - s->l_skip),
+                            num_sms());
+  pl.off_bytes = round_up(offset_bytes(g.units, g.rows), 256);
+  pl.part_bytes = pl.groups > 1 ? static_cast<size_t>(s->batch) * pl.n_blocks * pl.groups * s->hq * 256 * 4 : 0;
+  return pl;
+}
+
 size_t specpc_workspace_size(const spk_specpc_shape* s) {
   SpeckvGeom g;
   if (check_specpc(s, g) != SPK_OK) return 0;
-  return round_up(offset_bytes(g.units, g.rows), 256);
+  const SpecpcPlan pl = specpc_plan(s, g);
+  return pl.off_bytes + round_up(pl.part_bytes, 256);
+}
+
+static spk_status specpc_prepare(const spk_specpc_shape* s, const void* q, const void* k, const void* ws,
+                                 size_t ws_bytes, SpeckvGeom& g, CUtensorMap* qmap, CUtensorMap* kmap, ScoreParams& p) {
+  spk_status st = check_specpc(s, g);
+  if (st != SPK_OK) return st;
+  if (q == nullptr || k == nullptr) return fail(SPK_ERR_ARG, "q and k must be non-NULL device pointers");
+  if (!aligned16(q) || !aligned16(k)) return fail(SPK_ERR_ARG, "q and k must be 16-byte aligned");
+  const size_t need = specpc_workspace_size(s);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
+  const long long all_units = static_cast<long long>(s->batch) * s->layers * s->hkv;
+  if ((st = make_map(qmap, q, s->head_dim, g.rows, all_units)) != SPK_OK) return st;
+  if ((st = make_map(kmap, k, s->head_dim, s->n_in, all_units)) != SPK_OK) return st;
+  const int c0 = s->n_in + s->n_lookahead - s->n_rows;
+  p = base_params(s->head_dim, s->n_in, g, c0, s->scale, s->hkv, s->layers - s->l_skip, s->layers, s->l_skip);
+  p.off_blocks = static_cast<uint8_t*>(const_cast<void*>(ws));
+  p.off_tiles = static_cast<int>(row_tiles(g.rows));
+  p.seg_groups = 1;
+  return SPK_OK;
+}
+
+spk_status specpc_row_offsets(const spk_specpc_shape* s, const void* q, const void* k, const float* w, void* ws,
+                              size_t ws_bytes, void* stream) {
+  SpeckvGeom g;
+  CUtensorMap qmap, kmap;
+  ScoreParams p;
+  spk_status st = specpc_prepare(s, q, k, ws, ws_bytes, g, &qmap, &kmap, p);
+  if (st != SPK_OK) return st;
+  if (w == nullptr) return fail(SPK_ERR_ARG, "row_weights must be a non-NULL device pointer");
+  p.row_weights = w;
+  st = run_lse(p, qmap, kmap, s->head_dim, static_cast<cudaStream_t>(stream));
+  return st == SPK_OK ? ok() : st;
+}
+
+spk_status specpc_colsum(const spk_specpc_shape* s, const void* q, const void* k, float* scores, void* ws,
+                         size_t ws_bytes, void* stream) {
+  SpeckvGeom g;
+  CUtensorMap qmap, kmap;
+  ScoreParams p;
+  spk_status st = specpc_prepare(s, q, k, ws, ws_bytes, g, &qmap, &kmap, p);
+  if (st != SPK_OK) return st;
+  if (scores == nullptr) return fail(SPK_ERR_ARG, "scores must be a non-NULL device pointer");
+  const SpecpcPlan pl = specpc_plan(s, g);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  p.n_pre = s->n_in;
+  p.n_cols = s->n_in;
+  p.out0 = scores;
+  p.n_blocks = pl.n_blocks;
+  p.seg_groups = pl.groups;
+  p.part = pl.groups > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_bytes) : nullptr;
+  p.n_items = s->batch * pl.n_blocks * pl.groups;
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  cudaError_t e = launch_score(MODE_COLSUM_PC, s->head_dim, kmap, qmap, p, grid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "SpecPC column-sum launch");
+  if (pl.groups > 1) {
+    e = launch_specpc_merge(p.part, s->batch, s->n_in, pl.n_blocks, pl.groups, s->hq, scores, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "SpecPC merge launch");
+  }
+  return ok();
 }
 
 spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k, const float* w, float* scores,
@@ -258,33 +393,8 @@ spk_status specpc_score(const spk_specpc_shape* s, const void* q, const void* k,
   if (st != SPK_OK) return st;
   if (q == nullptr || k == nullptr || w == nullptr || scores == nullptr)
     return fail(SPK_ERR_ARG, "q, k, row_weights and scores must be non-NULL device pointers");
-  if (!aligned16(q) || !aligned16(k)) return fail(SPK_ERR_ARG, "q and k must be 16-byte aligned");
-  const size_t need = specpc_workspace_size(s);
-  if (ws == nullptr || ws_bytes < need)
-    return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
-  if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
-  const long long all_units = static_cast<long long>(s->batch) * s->layers * s->hkv;
-  CUtensorMap qmap, kmap;
-  if ((st = make_map(&qmap, q, s->head_dim, g.rows, all_units)) != SPK_OK) return st;
-  if ((st = make_map(&kmap, k, s->head_dim, s->n_in, all_units)) != SPK_OK) return st;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const int c0 = s->n_in + s->n_lookahead - s->n_rows;
-  ScoreParams p = base_params(s->head_dim, s->n_in, g, c0, s->scale, s->hkv, s->layers - s->l_skip, s->layers,
-                              s->l_skip);
-  p.off_blocks = static_cast<uint8_t*>(ws);
-  p.off_tiles = static_cast<int>(row_tiles(g.rows));
-  p.row_weights = w;
-  if ((st = run_lse(p, qmap, kmap, s->head_dim, cs)) != SPK_OK) return st;
-  p.row_weights = nullptr;
-  p.n_pre = s->n_in;
-  p.n_cols = s->n_in;
-  p.out0 = scores;
-  p.n_blocks = (s->n_in + 255) / 256;
-  p.n_items = s->batch * p.n_blocks;
-  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
-  cudaError_t e = launch_score(MODE_COLSUM_PC, s->head_dim, kmap, qmap, p, grid, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "SpecPC column-sum launch");
-  return ok();
+  if ((st = specpc_row_offsets(s, q, k, w, ws, ws_bytes, stream)) != SPK_OK) return st;
+  return specpc_colsum(s, q, k, scores, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ selection
@@ -293,10 +403,12 @@ size_t topk_workspace_size(int units, int n_cand) {
   return round_up(topk_ws_bytes(units, n_cand), 256);
 }
 
-spk_status topk_select(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail,
-                       int32_t* idx, float* pooled, void* ws, size_t ws_bytes, void* stream) {
+static spk_status topk_common(const float* scores, int units, int n_cand, int pool_mode, int pool_kernel, int k,
+                              int n_tail, int32_t* idx, float* pooled, void* ws, size_t ws_bytes, void* stream) {
   if (units < 0 || n_cand < 0 || k < 0 || n_tail < 0) return fail(SPK_ERR_ARG, "negative size");
   if (pool_kernel < 1 || (pool_kernel & 1) == 0) return fail(SPK_ERR_ARG, "pool_kernel must be odd and >= 1");
+  if (pool_mode != SPK_POOL_MAX && pool_mode != SPK_POOL_AVG)
+    return fail(SPK_ERR_ARG, "pool_mode must be SPK_POOL_MAX (0) or SPK_POOL_AVG (1), got %d", pool_mode);
   if (units == 0) return ok();
   const long long out_len = static_cast<long long>(k < n_cand ? k : n_cand) + n_tail;
   if (out_len > 0 && idx == nullptr) return fail(SPK_ERR_ARG, "idx must be non-NULL");
@@ -306,10 +418,20 @@ spk_status topk_select(const float* scores, int units, int n_cand, int pool_kern
     return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
   if (static_cast<long long>(units) > 0x7fffffffLL / (out_len > 0 ? out_len : 1) && out_len > 0)
     return fail(SPK_ERR_UNSUPPORTED, "output too large");
-  cudaError_t e = launch_topk(scores, units, n_cand, pool_kernel, k, n_tail, idx, pooled, ws,
+  cudaError_t e = launch_topk(scores, units, n_cand, pool_mode, pool_kernel, k, n_tail, idx, pooled, ws,
                               static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
   return ok();
+}
+
+spk_status topk_select(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail,
+                       int32_t* idx, float* pooled, void* ws, size_t ws_bytes, void* stream) {
+  return topk_common(scores, units, n_cand, SPK_POOL_MAX, pool_kernel, k, n_tail, idx, pooled, ws, ws_bytes, stream);
+}
+
+spk_status topk_select_pool(const float* scores, int units, int n_cand, int pool_mode, int pool_kernel, int k,
+                            int n_tail, int32_t* idx, float* pooled, void* ws, size_t ws_bytes, void* stream) {
+  return topk_common(scores, units, n_cand, pool_mode, pool_kernel, k, n_tail, idx, pooled, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ compaction

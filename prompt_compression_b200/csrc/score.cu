@@ -68,7 +68,9 @@ template <int MODE, int D>
 struct Cfg {
   static constexpr int kTileBytes = 128 * D * 2;          // 128 rows x D bf16
   static constexpr int kAtoms = D / 64;                    // 128-byte swizzle atoms along K
-  static constexpr int kAStages = (MODE == MODE_LSE) ? 1 : 2;
+  // The SpecPC column pass at head_dim 128 keeps one A stage: two stages
+  // (128 KB) next to the B ring and the per-head sums would exceed 227 KB.
+  static constexpr int kAStages = (MODE == MODE_LSE || (MODE == MODE_COLSUM_PC && D == 128)) ? 1 : 2;
   static constexpr int kBStages = (MODE == MODE_LSE) ? (D == 128 ? 4 : 8) : (D == 128 ? 2 : 4);
   static constexpr int kABytes = 2 * kTileBytes;
   static constexpr int kSmemA = kAStages * kABytes;
@@ -81,6 +83,7 @@ struct Cfg {
   static constexpr int kAccFloats = (MODE == MODE_COLSUM_PC) ? 2 * kHeadsMax * 256 : 0;
   static constexpr int kSmemBytes = 1024 + kSmemA + kSmemB + kOnesBytes + 4 * kAccFloats;
   static_assert(kBStageBytes % 1024 == 0, "B stages keep the 1024-byte alignment of the swizzled tiles");
+  static_assert(kSmemBytes <= 227 * 1024 - 4096, "dynamic shared memory (plus the static part) fits one CTA");
   // Pass 1 items are long (all keys of a unit): its A tiles live in TMEM and
   // the UMMAs read only B from shared memory; three accumulator buffers fill
   // the rest of TMEM.  The column passes change A every few steps: A stays in
@@ -92,18 +95,29 @@ struct Cfg {
 // Error sites: mode * 100 + role * 10 + barrier.
 __device__ __forceinline__ int site(int mode, int role, int which) { return mode * 100 + role * 10 + which; }
 
-__device__ __forceinline__ int n_segments(const ScoreParams& p, int mode) {
-  return mode == MODE_COLSUM_PC ? p.hkv * p.layers_used : 1;
+// Segments of an item: SpecPC walks the (KV head, layer) segments of its
+// batch element, split into p.seg_groups contiguous groups (item =
+// (key block) * seg_groups + group); the other modes have one segment.
+__device__ __forceinline__ int seg_begin(const ScoreParams& p, int mode, int item) {
+  if (mode != MODE_COLSUM_PC) return 0;
+  const int nseg = p.hkv * p.layers_used;
+  return static_cast<int>(static_cast<long long>(item % p.seg_groups) * nseg / p.seg_groups);
+}
+__device__ __forceinline__ int seg_end(const ScoreParams& p, int mode, int item) {
+  if (mode != MODE_COLSUM_PC) return 1;
+  const int nseg = p.hkv * p.layers_used;
+  return static_cast<int>(static_cast<long long>(item % p.seg_groups + 1) * nseg / p.seg_groups);
 }
 
 // (item, segment) -> unit, its 3-D tensor coordinate, first A row.
 __device__ __forceinline__ void decode(const ScoreParams& p, int mode, int item, int seg, int& u, int& tc,
                                        int& a_row0) {
   if (mode == MODE_COLSUM_PC) {
-    const int b = item / p.n_blocks;
+    const int blk = item / p.seg_groups;
+    const int b = blk / p.n_blocks;
     const int h = seg / p.layers_used, lu = seg % p.layers_used;
     u = (b * p.layers_used + lu) * p.hkv + h;
-    a_row0 = (item % p.n_blocks) * 256;
+    a_row0 = (blk % p.n_blocks) * 256;
   } else {
     u = item / p.n_blocks;
     a_row0 = (item % p.n_blocks) * 256;
@@ -319,7 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const uint32_t tmem_base = tmem_holder;
   volatile int* abort_v = &abort_flag;
-  const int nseg = n_segments(p, MODE);
   const int nb = b_tiles(p, MODE);
 
   if (warp == kProducerWarp) {
@@ -331,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int seg_count = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        for (int seg = 0; ok && seg < nseg; ++seg, ++seg_count) {
+        for (int seg = seg_begin(p, MODE, item); ok && seg < seg_end(p, MODE, item); ++seg, ++seg_count) {
           int u, tc, a_row0;
           decode(p, MODE, item, seg, u, tc, a_row0);
           if (!(ok = mbar_wait(&a_empty[a_stage], a_phase ^ 1, abort_v, site(MODE, 0, 0)))) break;
@@ -384,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint32_t a_tmem0 = tmem_base + 384;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        for (int seg = 0; ok && seg < nseg; ++seg, ++segs) {
+        for (int seg = seg_begin(p, MODE, item); ok && seg < seg_end(p, MODE, item); ++seg, ++segs) {
           int u, tc, a_row0;
           decode(p, MODE, item, seg, u, tc, a_row0);
           const bool act0 = a_tile_active(p, MODE, a_row0, 0);
@@ -526,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc_masked = 0.f;
       float m = -INFINITY, l = 0.f;                                                 // pass-1 row state
       int item_u = 0, item_row0 = 0;
-      for (int seg = 0; ok && seg < nseg; ++seg, ++seg_count) {
+      for (int seg = seg_begin(p, MODE, item); ok && seg < seg_end(p, MODE, item); ++seg, ++seg_count) {
         int u, tc, a_row0;
         decode(p, MODE, item, seg, u, tc, a_row0);
         item_u = u;
@@ -670,16 +683,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int row = item_row0 + r;
           if (a_tile_active(p, MODE, item_row0, t)) {
             float out = 0.f;
-            if (row < p.rows) {
+            bool live = row < p.rows;   // a row that contributes to the column sums
+            if (live) {
               const float M = fmaxf(m, m1);
               const float L = l * ex2_approx(m - M) + l1 * ex2_approx(m1 - M);
               out = M + lg2_approx(L);
-              if (p.row_weights != nullptr) out += log2_norm - log2f(p.row_weights[row % p.R]);
+              if (p.row_weights != nullptr) {
+                // weight w_i folds in as -log2(w_i); a row of weight 0 adds
+                // nothing and takes the padding offset (log2(0) = -inf would
+                // turn the three-term split into NaN)
+                const float w = p.row_weights[row % p.R];
+                if (w > 0.f) out += log2_norm - log2f(w);
+                else live = false;
+              }
             }
             if (p.off_blocks != nullptr) {
               if (row < p.off_tiles * 128)
                 store_offset_row(p.off_blocks + (static_cast<size_t>(item_u) * p.off_tiles + row / 128) * kOffBlockBytes,
-                                 row & 127, row < p.rows ? -out / p.c2 : -1e30f);
+                                 row & 127, live ? -out / p.c2 : -1e30f);
             } else if (row < p.rows) {
               p.lse2[static_cast<size_t>(item_u) * p.lse_stride + row] = out;
             }
@@ -708,18 +729,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           if (!(ok = wait_uniform(&mrg_full[0], items_done & 1, 1))) break;
           const int hq = (p.rows / p.R) * p.hkv;
-          float best = -INFINITY;
-          for (int qh = 0; qh < hq; ++qh) {
-            float* a0 = acc_s + qh * 256 + r;
-            float* a1 = acc_s + (kHeadsMax + qh) * 256 + r;
-            best = fmaxf(best, *a0 + *a1);
-            *a0 = 0.f;
-            *a1 = 0.f;
+          const int blk = item / p.seg_groups;
+          if (p.seg_groups == 1) {
+            float best = -INFINITY;
+            for (int qh = 0; qh < hq; ++qh) {
+              float* a0 = acc_s + qh * 256 + r;
+              float* a1 = acc_s + (kHeadsMax + qh) * 256 + r;
+              best = fmaxf(best, *a0 + *a1);
+              *a0 = 0.f;
+              *a1 = 0.f;
+            }
+            arrive_warp(&mrg_empty[0]);
+            const int b = blk / p.n_blocks;
+            const int j = (blk % p.n_blocks) * 256 + r;
+            if (j < p.n_cols) p.out0[static_cast<size_t>(b) * p.n_in + j] = best;
+          } else {
+            // this group's per-head partial sums; specpc_merge adds the
+            // groups in order and takes the head max
+            float* part = p.part + static_cast<size_t>(item) * hq * 256 + r;
+            for (int qh = 0; qh < hq; ++qh) {
+              float* a0 = acc_s + qh * 256 + r;
+              float* a1 = acc_s + (kHeadsMax + qh) * 256 + r;
+              part[qh * 256] = *a0 + *a1;
+              *a0 = 0.f;
+              *a1 = 0.f;
+            }
+            arrive_warp(&mrg_empty[0]);
           }
-          arrive_warp(&mrg_empty[0]);
-          const int b = item / p.n_blocks;
-          const int j = (item % p.n_blocks) * 256 + r;
-          if (j < p.n_cols) p.out0[static_cast<size_t>(b) * p.n_in + j] = best;
         }
       }
     }
@@ -734,6 +770,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+}
+
+// SpecPC with split segment groups: add each key's per-head partial sums over
+// the groups in group order, then take the max over query heads.  One thread
+// per key, 256 keys per block (consecutive threads read consecutive floats).
+__global__ void __launch_bounds__(256)
+    specpc_merge_kernel(const float* __restrict__ part, int n_in, int n_blocks, int groups, int hq,
+                        float* __restrict__ scores) {
+  const int blk = blockIdx.x;
+  const int r = threadIdx.x;
+  const int j = (blk % n_blocks) * 256 + r;
+  if (j >= n_in) return;
+  const float* base = part + static_cast<size_t>(blk) * groups * hq * 256 + r;
+  float best = -INFINITY;
+  for (int qh = 0; qh < hq; ++qh) {
+    float sum = 0.f;
+    for (int g = 0; g < groups; ++g) sum += base[(static_cast<size_t>(g) * hq + qh) * 256];
+    best = fmaxf(best, sum);
+  }
+  scores[static_cast<size_t>(blk / n_blocks) * n_in + j] = best;
+}
+
+cudaError_t launch_specpc_merge(const float* part, int batch, int n_in, int n_blocks, int groups, int hq,
+                                float* scores, cudaStream_t stream) {
+  specpc_merge_kernel<<<batch * n_blocks, 256, 0, stream>>>(part, n_in, n_blocks, groups, hq, scores);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -761,6 +823,7 @@ cudaError_t launch_score(int mode, int head_dim, const CUtensorMap& amap, const 
   if (head_dim == 128) {
     if (mode == MODE_LSE) return launch_one<MODE_LSE, 128>(amap, bmap, p, grid, stream);
     if (mode == MODE_COLSUM) return launch_one<MODE_COLSUM, 128>(amap, bmap, p, grid, stream);
+    if (mode == MODE_COLSUM_PC) return launch_one<MODE_COLSUM_PC, 128>(amap, bmap, p, grid, stream);
   } else if (head_dim == 64) {
     if (mode == MODE_LSE) return launch_one<MODE_LSE, 64>(amap, bmap, p, grid, stream);
     if (mode == MODE_COLSUM) return launch_one<MODE_COLSUM, 64>(amap, bmap, p, grid, stream);
@@ -773,6 +836,7 @@ int score_smem_bytes(int mode, int head_dim) {
   if (head_dim == 128) {
     if (mode == MODE_LSE) return Cfg<MODE_LSE, 128>::kSmemBytes;
     if (mode == MODE_COLSUM) return Cfg<MODE_COLSUM, 128>::kSmemBytes;
+    if (mode == MODE_COLSUM_PC) return Cfg<MODE_COLSUM_PC, 128>::kSmemBytes;
   } else {
     if (mode == MODE_LSE) return Cfg<MODE_LSE, 64>::kSmemBytes;
     if (mode == MODE_COLSUM) return Cfg<MODE_COLSUM, 64>::kSmemBytes;

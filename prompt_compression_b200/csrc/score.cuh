@@ -58,15 +58,28 @@ struct ScoreParams {
   int n_pre;         // prefix keys that are scored
   int n_cols;        // keys whose column sums are written
   const float* row_weights;  // SpecPC row weights [R] (LSE folds -log2(w_i / norm) into lse2)
+  // SpecPC column pass: the (KV head, layer) segments of a key block are
+  // split into seg_groups groups (one item each); with more than one group
+  // every item writes per-query-head partial sums [item][hq][256] to part,
+  // and launch_specpc_merge reduces them.
+  int seg_groups;
+  float* part;
 };
 
 cudaError_t launch_score(int mode, int head_dim, const CUtensorMap& amap, const CUtensorMap& bmap,
                          const ScoreParams& p, int grid, cudaStream_t stream);
+// scores[b][j] = max_qh sum_g part[(b * n_blocks + j / 256) * groups + g][qh][j % 256]
+cudaError_t launch_specpc_merge(const float* part, int batch, int n_in, int n_blocks, int groups, int hq,
+                                float* scores, cudaStream_t stream);
 int score_smem_bytes(int mode, int head_dim);
 
 // pooling + top-k selection (select.cu)
-cudaError_t launch_topk(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail,
-                        int* idx, float* pooled, void* ws, cudaStream_t stream);
+enum PoolMode : int {
+  POOL_MAX = 0,   // max over the clipped window
+  POOL_AVG = 1,   // sum over the clipped window / its length
+};
+cudaError_t launch_topk(const float* scores, int units, int n_cand, int pool_mode, int pool_kernel, int k,
+                        int n_tail, int* idx, float* pooled, void* ws, cudaStream_t stream);
 size_t topk_ws_bytes(int units, int n_cand);
 
 // row gather (compact.cu)

@@ -1,21 +1,32 @@
-// select.cu -- max-pooling and deterministic top-k selection with a kept tail.
+// select.cu -- local pooling and deterministic top-k selection with a kept tail.
 //
 // "Draft-based Approximate Inference for LLMs" (paper notes): section 关键设计
 // keeps the top-C_max KV pairs plus the window; section 损失函数 / 训练策略
 // smooths SpecPC scores with local pooling so that kept tokens form runs.
+// The pages name local pooling without its kind: max pooling (the workloads'
+// "pool 7") and average pooling (mean over the clipped window) are offered.
 //
-// One CTA (512 threads) per row of candidates:
-//   1. pooled[j] = max of scores over the clipped window [j-r, j+r]: tiles of
-//      scores with their halo are staged in shared memory (coalesced loads);
-//      the pooled values are stored as order-preserving 32-bit keys, and a
-//      4096-bin histogram of their top 12 bits is built on the way.
-//   2. radix select in three passes (12, 12 and 8 bits, most significant
-//      first) finds the exact key T of the C-th largest value and how many
-//      keys equal to T must be taken; histogram updates are warp-aggregated.
-//   3. emission: each warp owns a contiguous run of indices and walks it 32
-//      at a time with ballots; one prefix over the warps' counts (keys equal
-//      to T, then selected keys) gives every warp its output offset, so the
-//      indices come out ascending with ties resolved lowest index first.
+// One CTA (512 threads) per row of candidates.  Pooled values are turned into
+// order-preserving 32-bit keys (a larger float gives a larger key).
+//   1. sweep 1: tiles of 2048 scores plus the pooling halo are staged in
+//      shared memory (five independent loads per thread in flight); every
+//      pooled value is formed there and counted in a 4096-bin histogram of
+//      its key's top 12 bits.  The bin B1 that holds the C-th largest key
+//      follows from one scan of the histogram.
+//   2. sweep 2 forms the same pooled values again (the same fp32 operations,
+//      so the same keys): keys in bins above B1 are selected outright and
+//      their indices collected; keys in B1 are collected with their index as
+//      candidates.  Both lists live in shared memory.
+//   3. the candidates are sorted by (key descending, index ascending), the
+//      first C - |selected| of them complete the selection, and the C indices
+//      are sorted ascending: ties go to the lower index, the output is
+//      ordered, and the result does not depend on the order in which threads
+//      appended to the lists.
+// When C exceeds 2048, or more than 2048 candidates share bin B1 (long runs of
+// equal values), a general path takes over: the keys go to the workspace and
+// a three-level radix select (12 + 12 + 8 bits) finds the exact C-th key T;
+// an ordered ballot walk over each warp's contiguous share of the row emits
+// the indices ascending, keys equal to T lowest index first.
 #include "common.cuh"
 #include "score.cuh"
 
@@ -25,7 +36,10 @@ namespace {
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kBins = 4096;
-constexpr int kHaloMax = kSelThreads;   // pooling radius staged through shared memory
+constexpr int kTile = 2048;                 // candidates per staged tile
+constexpr int kHaloMax = 256;               // pooling radius served from the staged tile
+constexpr int kTileLoads = (kTile + 2 * kHaloMax + kSelThreads - 1) / kSelThreads;   // 5
+constexpr int kListMax = 2048;              // shared-memory selection lists
 
 // Monotone map from finite floats to uint32 (larger float -> larger key);
 // -0 is folded onto +0 so that the two compare equal, as they do as floats.
@@ -72,7 +86,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
 
 // Given the histogram of the candidates that still match the prefix, find
 // the bin holding the remaining-th largest: bins are scanned from the top,
-// kBins / kSelThreads consecutive bins per thread.  Returns the bin (in
+// nbins / kSelThreads consecutive bins per thread.  Returns the bin (in
 // s_bin) and the count still to take inside it (in s_rem).
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int remaining, int* warp_tot,
                                          int* s_bin, int* s_rem) {
@@ -98,73 +112,138 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int re
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelThreads, 4)
-    topk_kernel(const float* __restrict__ scores, int n_cand, int pool_r, int k, int n_tail, int* __restrict__ idx,
-                float* __restrict__ pooled, uint32_t* __restrict__ keys_ws) {
-  __shared__ uint32_t hist[kBins];
-  __shared__ float tile[kSelThreads + 2 * kHaloMax];
-  __shared__ int warp_tot[33];
-  __shared__ int s_bin, s_rem;
-
-  const int u = blockIdx.x;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int n = n_cand;
-  const int C = k < n ? k : n;
-  const size_t out_len = static_cast<size_t>(C) + n_tail;
-  int* out = idx + static_cast<size_t>(u) * out_len;
-
-  // kept tail (the window)
-  for (int t = tid; t < n_tail; t += kSelThreads) out[C + t] = n + t;
-  if (C == 0 && pooled == nullptr) return;
-
-  const float* s = scores + static_cast<size_t>(u) * n;
-  uint32_t* keys = keys_ws + static_cast<size_t>(u) * n;
-  float* pout = pooled ? pooled + static_cast<size_t>(u) * n : nullptr;
-
-  // 1. pooling -> keys, histogram of the top 12 bits
-  for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0;
-  __syncthreads();
-  const bool staged = pool_r <= kHaloMax;
-  for (int base = 0; base < n; base += kSelThreads) {
-    const int j = base + tid;
+// Pooled value of candidate j.  `w` points at scores[j - r] inside a staged
+// tile whose slots outside [0, n) hold the padding (-inf for max, 0 for the
+// average), so the window needs no bounds tests.  The average divides the
+// sum of the clipped window (in window order) by its length.
+__device__ __forceinline__ float pool_staged(const float* w, int r, int mode, int j, int n) {
+  if (mode == POOL_MAX) {
     float m = -INFINITY;
+    for (int t = 0; t <= 2 * r; ++t) m = fmaxf(m, w[t]);
+    return m;
+  }
+  float s = 0.f;
+  for (int t = 0; t <= 2 * r; ++t) s += w[t];
+  const int lo = j - r < 0 ? 0 : j - r;
+  const int hi = j + r > n - 1 ? n - 1 : j + r;
+  return __fdiv_rn(s, static_cast<float>(hi - lo + 1));
+}
+
+// The same value read straight from global memory (radii beyond the halo).
+__device__ __forceinline__ float pool_direct(const float* s, int r, int mode, int j, int n) {
+  const int lo = j - r < 0 ? 0 : j - r;
+  const int hi = j + r > n - 1 ? n - 1 : j + r;
+  if (mode == POOL_MAX) {
+    float m = -INFINITY;
+    for (int t = lo; t <= hi; ++t) m = fmaxf(m, s[t]);
+    return m;
+  }
+  float acc = 0.f;
+  for (int t = lo; t <= hi; ++t) acc += s[t];
+  return __fdiv_rn(acc, static_cast<float>(hi - lo + 1));
+}
+
+// Calls f(j, valid, pooled_j) for every candidate j of the row, warp-uniformly
+// (every lane of every warp calls f the same number of times; lanes past the
+// end pass valid = false), tile by tile.
+template <typename F>
+__device__ __forceinline__ void pooled_sweep(const float* __restrict__ s, int n, int r, int mode, float* tile,
+                                             F&& f) {
+  const int tid = threadIdx.x;
+  const bool staged = r <= kHaloMax;
+  const float pad = mode == POOL_MAX ? -INFINITY : 0.f;
+  for (int base = 0; base < n; base += kTile) {
     if (staged) {
-      // scores[base - r, base + kSelThreads + r) with -inf outside [0, n):
-      // the max over the padded window equals the max over the clipped one
-      for (int t = tid; t < kSelThreads + 2 * pool_r; t += kSelThreads) {
-        const int jj = base - pool_r + t;
-        tile[t] = (jj >= 0 && jj < n) ? s[jj] : -INFINITY;
+      // scores[base - r, base + kTile + r) with padding outside [0, n): all
+      // loads of a thread are issued before any of them is stored
+      const int len = kTile + 2 * r;
+      float v[kTileLoads];
+#pragma unroll
+      for (int q = 0; q < kTileLoads; ++q) {
+        const int t = tid + q * kSelThreads;
+        const int jj = base - r + t;
+        v[q] = (t < len && jj >= 0 && jj < n) ? __ldg(s + jj) : pad;
+      }
+#pragma unroll
+      for (int q = 0; q < kTileLoads; ++q) {
+        const int t = tid + q * kSelThreads;
+        if (t < len) tile[t] = v[q];
       }
       __syncthreads();
-      if (j < n)
-        for (int t = 0; t <= 2 * pool_r; ++t) m = fmaxf(m, tile[tid + t]);
-      __syncthreads();
-    } else if (j < n) {
-      const int lo = j - pool_r < 0 ? 0 : j - pool_r;
-      const int hi = j + pool_r > n - 1 ? n - 1 : j + pool_r;
-      for (int t = lo; t <= hi; ++t) m = fmaxf(m, s[t]);
     }
+#pragma unroll 1
+    for (int i = 0; i < kTile / kSelThreads; ++i) {
+      const int off = i * kSelThreads + tid;
+      const int j = base + off;
+      const bool valid = j < n;
+      float p = 0.f;
+      if (valid) p = staged ? pool_staged(tile + off, r, mode, j, n) : pool_direct(s, r, mode, j, n);
+      f(j, valid, p);
+    }
+    if (staged) __syncthreads();
+  }
+}
+
+// Ascending bitonic sort of a[0, P) in shared memory, P a power of two.
+template <typename T>
+__device__ __forceinline__ void bitonic_sort(T* a, int P) {
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < P; i += kSelThreads) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const T x = a[i], y = a[ixj];
+          const bool up = (i & k) == 0;
+          if ((x > y) == up) {
+            a[i] = y;
+            a[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__device__ __forceinline__ int pow2_at_least(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+struct SelShared {
+  float tile[kTile + 2 * kHaloMax];
+  union {
+    uint32_t hist[kBins];
+    unsigned long long cand[kListMax];   // (~key << 32) | index: ascending = key desc, index asc
+  } u;
+  int list[kListMax];
+  int warp_tot[33];
+  int s_bin, s_rem, n_a, n_b;
+};
+
+// General path (C > kListMax, or too many candidates in the threshold bin):
+// keys in the workspace, three radix levels, ordered ballot emission.
+__device__ __noinline__ void select_general(SelShared& sh, const float* __restrict__ s, int n, int r, int mode,
+                                            int C, uint32_t* __restrict__ keys, int* __restrict__ out) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  uint32_t* hist = sh.u.hist;
+  for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0;
+  __syncthreads();
+  pooled_sweep(s, n, r, mode, sh.tile, [&](int j, bool valid, float p) {
     uint32_t bin = kBins;
-    if (j < n) {
-      if (pout) pout[j] = m;
-      const uint32_t key = float_key(m);
+    if (valid) {
+      const uint32_t key = float_key(p);
       keys[j] = key;
       bin = key >> 20;
     }
     hist_add(hist, bin);
-  }
-  if (C == 0) return;
-  if (C >= n) {
-    for (int j = tid; j < n; j += kSelThreads) out[j] = j;
-    return;
-  }
+  });
   __syncthreads();
-
-  // 2. radix select: 12 + 12 + 8 bits
-  find_bin(hist, kBins, C, warp_tot, &s_bin, &s_rem);
-  uint32_t prefix = static_cast<uint32_t>(s_bin);        // top 12 bits of T
-  int remaining = s_rem;
+  find_bin(hist, kBins, C, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  uint32_t prefix = static_cast<uint32_t>(sh.s_bin);        // top 12 bits of T
+  int remaining = sh.s_rem;
   for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0;
   __syncthreads();
   for (int base = 0; base < n; base += kSelThreads) {
@@ -177,9 +256,9 @@ __global__ void __launch_bounds__(kSelThreads, 4)
     hist_add(hist, bin);
   }
   __syncthreads();
-  find_bin(hist, kBins, remaining, warp_tot, &s_bin, &s_rem);
-  prefix = (prefix << 12) | static_cast<uint32_t>(s_bin);   // top 24 bits of T
-  remaining = s_rem;
+  find_bin(hist, kBins, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  prefix = (prefix << 12) | static_cast<uint32_t>(sh.s_bin);   // top 24 bits of T
+  remaining = sh.s_rem;
   for (int b = tid; b < 256; b += kSelThreads) hist[b] = 0;
   __syncthreads();
   for (int base = 0; base < n; base += kSelThreads) {
@@ -192,11 +271,11 @@ __global__ void __launch_bounds__(kSelThreads, 4)
     hist_add(hist, bin);
   }
   __syncthreads();
-  find_bin(hist, 256, remaining, warp_tot, &s_bin, &s_rem);
-  const uint32_t T = (prefix << 8) | static_cast<uint32_t>(s_bin);
-  const int take_eq = s_rem;   // keys equal to T to take, lowest index first
+  find_bin(hist, 256, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  const uint32_t T = (prefix << 8) | static_cast<uint32_t>(sh.s_bin);
+  const int take_eq = sh.s_rem;   // keys equal to T to take, lowest index first
 
-  // 3. ordered emission: warp w owns [w * chunk, (w + 1) * chunk)
+  // ordered emission: warp w owns [w * chunk, (w + 1) * chunk)
   const int chunk = ((n + kSelWarps - 1) / kSelWarps + 31) & ~31;
   const int beg = warp * chunk < n ? warp * chunk : n;
   const int end = beg + chunk < n ? beg + chunk : n;
@@ -209,10 +288,10 @@ __global__ void __launch_bounds__(kSelThreads, 4)
   }
   int total;
   // one value per warp: lane 0 carries it, the others add nothing
-  const int eq_before = __shfl_sync(0xffffffffu, block_exclusive_scan(lane == 0 ? eq : 0, warp_tot, total), 0);
+  const int eq_before = __shfl_sync(0xffffffffu, block_exclusive_scan(lane == 0 ? eq : 0, sh.warp_tot, total), 0);
   int my_eq = take_eq - eq_before;
   my_eq = my_eq < 0 ? 0 : (my_eq > eq ? eq : my_eq);
-  int pos = __shfl_sync(0xffffffffu, block_exclusive_scan(lane == 0 ? gt + my_eq : 0, warp_tot, total), 0);
+  int pos = __shfl_sync(0xffffffffu, block_exclusive_scan(lane == 0 ? gt + my_eq : 0, sh.warp_tot, total), 0);
   const uint32_t lt_mask = (1u << lane) - 1u;
   for (int j0 = beg; j0 < end; j0 += 32) {
     const int j = j0 + lane;
@@ -227,17 +306,109 @@ __global__ void __launch_bounds__(kSelThreads, 4)
   }
 }
 
+__global__ void __launch_bounds__(kSelThreads, 4)
+    topk_kernel(const float* __restrict__ scores, int n_cand, int pool_r, int pool_mode, int k, int n_tail,
+                int* __restrict__ idx, float* __restrict__ pooled, uint32_t* __restrict__ keys_ws) {
+  __shared__ SelShared sh;
+  const int u = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int n = n_cand;
+  const int C = k < n ? k : n;
+  const size_t out_len = static_cast<size_t>(C) + n_tail;
+  int* out = idx + static_cast<size_t>(u) * out_len;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  // kept tail (the window)
+  for (int t = tid; t < n_tail; t += kSelThreads) out[C + t] = n + t;
+  if (C == 0 && pooled == nullptr) return;
+
+  const float* s = scores + static_cast<size_t>(u) * n;
+  uint32_t* keys = keys_ws + static_cast<size_t>(u) * n;
+  float* pout = pooled ? pooled + static_cast<size_t>(u) * n : nullptr;
+
+  // 1. pooled values -> (optional output) and the histogram of the keys' top 12 bits
+  for (int b = tid; b < kBins; b += kSelThreads) sh.u.hist[b] = 0;
+  if (tid == 0) { sh.n_a = 0; sh.n_b = 0; }
+  __syncthreads();
+  pooled_sweep(s, n, pool_r, pool_mode, sh.tile, [&](int j, bool valid, float p) {
+    uint32_t bin = kBins;
+    if (valid) {
+      if (pout) pout[j] = p;
+      bin = float_key(p) >> 20;
+    }
+    if (C > 0 && C < n) hist_add(sh.u.hist, bin);
+  });
+  if (C == 0) return;
+  if (C >= n) {
+    for (int j = tid; j < n; j += kSelThreads) out[j] = j;
+    return;
+  }
+  if (C > kListMax) {
+    __syncthreads();             // every thread is done with sweep 1's histogram
+    select_general(sh, s, n, pool_r, pool_mode, C, keys, out);
+    return;
+  }
+  __syncthreads();
+  find_bin(sh.u.hist, kBins, C, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  const uint32_t b1 = static_cast<uint32_t>(sh.s_bin);
+  const int need = sh.s_rem;     // keys of bin b1 still to take (>= 1)
+  __syncthreads();               // everyone has read the histogram: its memory now holds candidates
+
+  // 2. bins above b1 are selected; bin b1 holds the candidates
+  pooled_sweep(s, n, pool_r, pool_mode, sh.tile, [&](int j, bool valid, float p) {
+    const uint32_t key = valid ? float_key(p) : 0u;
+    const uint32_t bin = key >> 20;
+    const bool is_a = valid && bin > b1;
+    const bool is_b = valid && bin == b1;
+    const uint32_t ma = __ballot_sync(0xffffffffu, is_a);
+    const uint32_t mb = __ballot_sync(0xffffffffu, is_b);
+    int base_a = 0, base_b = 0;
+    if (lane == 0) {
+      if (ma) base_a = atomicAdd(&sh.n_a, __popc(ma));
+      if (mb) base_b = atomicAdd(&sh.n_b, __popc(mb));
+    }
+    base_a = __shfl_sync(0xffffffffu, base_a, 0);
+    base_b = __shfl_sync(0xffffffffu, base_b, 0);
+    if (is_a) sh.list[base_a + __popc(ma & lt_mask)] = j;   // fewer than C <= kListMax of these
+    if (is_b) {
+      const int pos = base_b + __popc(mb & lt_mask);
+      if (pos < kListMax)
+        sh.u.cand[pos] = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(j);
+    }
+  });
+  __syncthreads();
+  const int n_a = sh.n_a, n_b = sh.n_b;
+  if (n_b > kListMax) {          // a long run of (nearly) equal values: the general path
+    __syncthreads();
+    select_general(sh, s, n, pool_r, pool_mode, C, keys, out);
+    return;
+  }
+
+  // 3. order the candidates, complete the selection, order the indices
+  const int pb = pow2_at_least(n_b);
+  for (int t = n_b + tid; t < pb; t += kSelThreads) sh.u.cand[t] = ~0ull;
+  __syncthreads();
+  bitonic_sort(sh.u.cand, pb);
+  for (int t = tid; t < need; t += kSelThreads) sh.list[n_a + t] = static_cast<int>(sh.u.cand[t] & 0xffffffffu);
+  const int pc = pow2_at_least(C);
+  for (int t = C + tid; t < pc; t += kSelThreads) sh.list[t] = 0x7fffffff;
+  __syncthreads();
+  bitonic_sort(sh.list, pc);
+  for (int t = tid; t < C; t += kSelThreads) out[t] = sh.list[t];
+}
+
 }  // namespace
 
 size_t topk_ws_bytes(int units, int n_cand) {
   return static_cast<size_t>(units) * static_cast<size_t>(n_cand > 0 ? n_cand : 0) * sizeof(uint32_t);
 }
 
-cudaError_t launch_topk(const float* scores, int units, int n_cand, int pool_kernel, int k, int n_tail, int* idx,
-                        float* pooled, void* ws, cudaStream_t stream) {
+cudaError_t launch_topk(const float* scores, int units, int n_cand, int pool_mode, int pool_kernel, int k,
+                        int n_tail, int* idx, float* pooled, void* ws, cudaStream_t stream) {
   if (units == 0) return cudaSuccess;
-  topk_kernel<<<units, kSelThreads, 0, stream>>>(scores, n_cand, pool_kernel / 2, k, n_tail, idx, pooled,
-                                                 static_cast<uint32_t*>(ws));
+  topk_kernel<<<units, kSelThreads, 0, stream>>>(scores, n_cand, pool_kernel / 2, pool_mode, k, n_tail, idx,
+                                                 pooled, static_cast<uint32_t*>(ws));
   return cudaGetLastError();
 }
 

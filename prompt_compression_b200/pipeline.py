@@ -42,17 +42,19 @@ class SpeckvBuffers:
 
 
 def speckv_compress(q, k, v, n_window: int, c_max: int, pool: int = 7, scale: float = 1.0,
-                    buffers: Optional[SpeckvBuffers] = None, window_mass: bool = False, stream=None):
-    """SpecKV on every unit: returns the buffers object (scores, idx, k_out, v_out)."""
+                    buffers: Optional[SpeckvBuffers] = None, window_mass: bool = False, stream=None,
+                    pool_mode: int = B.SPK_POOL_MAX):
+    """SpecKV on every unit: returns the buffers object (scores, idx, k_out, v_out).
+    pool_mode: B.SPK_POOL_MAX (the workloads' max pool) or B.SPK_POOL_AVG."""
     buf = buffers or SpeckvBuffers(q, k, v, n_window, c_max, window_mass=window_mass)
     B.speckv_score(q, k, n_window, buf.scores, buf.window_mass, buf.ws_score, scale, stream)
-    B.topk_select(buf.scores, c_max, n_window, buf.idx, pool, buf.pooled, buf.ws_topk, stream)
+    B.topk_select(buf.scores, c_max, n_window, buf.idx, pool, buf.pooled, buf.ws_topk, stream, pool_mode)
     B.kv_compact(k, v, buf.idx, buf.k_out, buf.v_out, 1, stream)
     return buf
 
 
 def specpc_select(q, k, row_weights, l_skip: int, keep: int, pool: int = 7, n_lookahead: int = 1,
-                  scale: float = 1.0, scores=None, idx=None, stream=None):
+                  scale: float = 1.0, scores=None, idx=None, stream=None, pool_mode: int = B.SPK_POOL_MAX):
     """SpecPC prompt-token selection: (scores [B, n_in], idx [B, min(keep, n_in)])."""
     Bsz = q.shape[0]
     n_in = k.shape[3]
@@ -61,7 +63,7 @@ def specpc_select(q, k, row_weights, l_skip: int, keep: int, pool: int = 7, n_lo
     if idx is None:
         idx = torch.empty((Bsz, min(keep, n_in)), dtype=torch.int32, device=q.device)
     B.specpc_score(q, k, row_weights, scores, l_skip, n_lookahead, None, scale, stream)
-    B.topk_select(scores, keep, 0, idx, pool, None, None, stream)
+    B.topk_select(scores, keep, 0, idx, pool, None, None, stream, pool_mode)
     return scores, idx
 
 

@@ -26,7 +26,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for f in ("speckv_score", "specpc_score", "topk_select", "kv_compact", "spk_last_error",
+    for f in ("speckv_score", "specpc_score", "topk_select", "topk_select_pool", "kv_compact", "spk_last_error",
               "speckv_workspace_size", "specpc_workspace_size", "topk_workspace_size"):
         assert f in names
 
@@ -41,7 +41,11 @@ def test_workspace_sizes(lib):
     s = B.SpeckvShape(1, 64, 40, 8, 128, 65536, 64, 128, 1.0)
     assert B.speckv_workspace_size(s) == 512 * 1024 * 32    # 32 B per row, rows padded to 128
     s = B.SpecpcShape(1, 24, 4, 14, 2, 64, 32768, 256, 1, 1.0)
-    assert B.specpc_workspace_size(s) == 40 * 1792 * 32
+    # row offsets (40 units x 1792 rows x 32 B) + on 148 SMs the 128 key blocks
+    # are split into 8 segment groups: 128 x 8 x 14 heads x 1 KB of partial sums
+    assert B.specpc_workspace_size(s) == 40 * 1792 * 32 + 128 * 8 * 14 * 1024
+    s = B.SpecpcShape(2, 24, 4, 14, 2, 64, 131072, 256, 1, 1.0)
+    assert B.specpc_workspace_size(s) == 80 * 1792 * 32      # 1024 blocks fill 148 SMs: no split
     assert B.topk_workspace_size(512, 65472) == 512 * 65472 * 4
 
 
@@ -73,7 +77,7 @@ def test_speckv_workspace_and_pointer_errors(lib):
 def test_specpc_argument_errors(lib):
     from prompt_compression_b200 import binding as B
     bad = [((1, 4, 4, 4, 2, 64, 100, 16, 1, 1.0), 1),      # l_skip == layers
-           ((1, 4, 1, 4, 2, 128, 100, 16, 1, 1.0), 2),     # head_dim 128 unsupported
+           ((1, 4, 1, 4, 2, 96, 100, 16, 1, 1.0), 2),      # head_dim 96 unsupported
            ((1, 4, 1, 4, 2, 64, 100, 101, 1, 1.0), 1),     # window longer than the input
            ((1, 4, 1, 34, 2, 64, 100, 16, 1, 1.0), 2),     # group of 17 query heads
            ((1, 4, 1, 4, 2, 64, 100, 16, 0, 1.0), 1)]      # no lookahead token
@@ -87,6 +91,9 @@ def test_topk_and_compact_argument_errors(lib):
     assert lib.topk_select(16, 4, 100, 4, 10, 0, 16, None, 16, 1 << 20, None) == B.SPK_ERR_ARG  # even pool
     assert lib.topk_select(16, 4, 100, 7, 10, 0, 16, None, 16, 8, None) == B.SPK_ERR_WORKSPACE
     assert lib.topk_select(16, 4, 100, 7, -1, 0, 16, None, 16, 1 << 20, None) == B.SPK_ERR_ARG
+    assert lib.topk_select_pool(16, 4, 100, 2, 7, 10, 0, 16, None, 16, 1 << 20, None) == B.SPK_ERR_ARG   # mode
+    assert "pool_mode" in lib.spk_last_error().decode()
+    assert lib.topk_select_pool(16, 4, 100, 1, 6, 10, 0, 16, None, 16, 1 << 20, None) == B.SPK_ERR_ARG   # even
     assert lib.kv_compact(16, 16, 4, 10, 60, 2, 16, 3, 1, 16, 16, None) == B.SPK_ERR_UNSUPPORTED
     assert lib.kv_compact(16, 16, 5, 10, 64, 2, 16, 3, 2, 16, 16, None) == B.SPK_ERR_ARG
     assert lib.kv_compact(16, None, 4, 10, 64, 2, 16, 3, 1, 16, 16, None) == B.SPK_ERR_ARG

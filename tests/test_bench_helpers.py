@@ -5,11 +5,15 @@ import json
 import bench
 
 
-def test_tensor_peak_prefers_the_sustained_figure():
+def test_tensor_peak_is_the_burst_figure():
+    # kernels are timed per launch (milliseconds), so the burst GEMM figure
+    # is the denominator; the sustained one is context only
     peak, src = bench.tensor_peak({"bf16_tflops": 1615.5, "bf16_tflops_sustained": 1379.5, "source": "measured"})
-    assert peak == 1379.5 and "sustained" in src
-    peak, src = bench.tensor_peak({"bf16_tflops": 1615.5, "bf16_tflops_sustained": None, "source": "measured"})
     assert peak == 1615.5 and "burst" in src
+    r = bench.kernel_roofline("k", 10.0, 8.0e12, {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
+                                                 "hbm_gbs": 6500.0, "source": "measured"})
+    assert abs(r["achieved"] - 800.0) < 1e-9 and abs(r["frac"] - 0.5) < 1e-12
+    assert abs(r["frac_of_sustained"] - 800.0 / 1400.0) < 1e-12
 
 
 def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
@@ -37,3 +41,32 @@ def test_digest_covers_the_scoring_sources_only():
 def test_exp2_peak_from_unit_counts():
     # 148 SMs x (16 MUFU / (1 - 0.4 polynomial share)) per clock x 1965 MHz
     assert abs(bench.exp2_peak_per_s() - 148 * 16 / 0.6 * 1965e6) < 1.0
+
+
+def test_suite_names_resolve():
+    for name in bench.SUITE:
+        cfg = bench.config_of(name)
+        assert cfg is not None
+    assert bench.config_of("qwen2.5-32b_speckv_64k@2048").c_max == 2048
+
+
+def test_cpu_baselines_on_tiny_workloads():
+    # the oracle-timing plumbing: spawned processes draw their own inputs and
+    # report oracle seconds; the value is the timed work over (CPU-s / cores)
+    import dataclasses
+    import workloads as W
+    full = bench.cpu_baseline_speckv(W.TINY, 0, 2, full=True)
+    assert full["kind"] == "oracle" and full["cores"] == 2 and full["value"] > 0
+    cfg = dataclasses.replace(W.TINY, layers=2)
+    part = bench.cpu_baseline_speckv(cfg, 0, 2)
+    assert part["value"] > 0 and "1 of its 2 query heads" in part["sample"]
+    pc = W.SpecPCConfig("tiny_pc", batch=1, layers=3, l_skip=1, hq=4, hkv=2, head_dim=64, n_in=300,
+                        n_rows=32, n_lookahead=1, keep=40)
+    r = bench.cpu_baseline_specpc(pc, 0, 2)
+    assert r["value"] > 0 and "2 (batch, layer)" in r["sample"]
+    cc = W.CascadeConfig("tiny_cascade", draft=dataclasses.replace(pc, batch=2, keep=96),
+                         target=W.SpecKVConfig("t", batch=2, layers=1, hq=4, hkv=2, head_dim=64, n_in=96,
+                                               n_window=8, n_lookahead=8, c_max=16),
+                         n_in_full=300)
+    r = bench.cpu_baseline_cascade(cc, 0, 2)
+    assert r["value"] > 0 and "extrapolated" in r["sample"]

@@ -156,6 +156,24 @@ def test_deterministic(P):
     assert torch.equal(sa, b.scores) and torch.equal(ia, b.idx) and torch.equal(ka, b.k_out)
 
 
+def test_split_passes_equal_speckv_score(P):
+    # speckv_score is speckv_row_offsets then speckv_colsum: bit for bit
+    import torch
+    qb, kb, vb = _random_case(29, 1, 2, 8, 2, 128, 1300, 32, 64)
+    q, k = to_bf16_tensor(qb), to_bf16_tensor(kb)
+    units, n_pre = 4, 1300 - 32
+    a = torch.empty((units, n_pre), dtype=torch.float32, device="cuda")
+    wa = torch.empty((units, 32), dtype=torch.float32, device="cuda")
+    P.speckv_score(q, k, 32, a, wa)
+    ws = torch.empty(P.speckv_workspace_size(P.binding.speckv_shape(q, k, 32)), dtype=torch.uint8, device="cuda")
+    b = torch.full_like(a, float("nan"))
+    wb = torch.full_like(wa, float("nan"))
+    P.speckv_row_offsets(q, k, 32, ws)
+    P.speckv_colsum(q, k, 32, b, ws, window_mass=wb)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(wa, wb)
+
+
 def test_uniform_keys_ties_lowest_index(P):
     # identical keys: all prefix scores tie exactly -> indices 0..C-1
     import torch
@@ -188,6 +206,60 @@ def test_topk_select_direct(P):
             ref = oracle.topk_with_tail(oracle.maxpool(s[u].astype(np.float64), pool) if n else
                                         np.zeros(0), kk, tail)
             assert got[u].tolist() == ref.tolist(), (n, kk, tail, pool)
+
+
+@pytest.mark.parametrize("mode", ["max", "avg"])
+def test_topk_paths_on_continuous_scores(P, mode):
+    """Both selection paths on continuous scores: the shared-memory path (C up
+    to 2048 with few candidates in the threshold bin) and the general radix
+    path (C above 2048), with either pooling; bit-exact against the oracle's
+    selection on the GPU's own pooled values, which match the oracle's
+    pooling of the GPU's scores (max: exactly; avg: fp32 sums, 1e-6)."""
+    import torch
+    rng = np.random.default_rng(19)
+    pm = P.SPK_POOL_MAX if mode == "max" else P.SPK_POOL_AVG
+    for n, kk, tail, pool in [(65472, 256, 64, 7), (65472, 2048, 0, 7), (65472, 2049, 0, 7),
+                              (20000, 5000, 3, 3), (777, 1, 2, 9), (777, 776, 0, 1), (4096, 300, 0, 1023)]:
+        s = (rng.gamma(2.0, 1.0, size=(3, n)) * rng.random((3, 1))).astype(np.float32)
+        st = torch.from_numpy(s).cuda()
+        c = min(kk, n)
+        idx = torch.empty((3, c + tail), dtype=torch.int32, device="cuda")
+        pooled = torch.empty((3, n), dtype=torch.float32, device="cuda")
+        P.topk_select(st, kk, tail, idx, pool, pooled=pooled, pool_mode=pm)
+        torch.cuda.synchronize()
+        got, gp = idx.cpu().numpy(), pooled.cpu().numpy()
+        for u in range(3):
+            ref_pool = oracle.pool(s[u].astype(np.float64), pool, mode)
+            if mode == "max":
+                np.testing.assert_array_equal(gp[u], ref_pool.astype(np.float32))
+            else:
+                np.testing.assert_allclose(gp[u], ref_pool, rtol=1e-6, atol=0)
+            own = oracle.topk_with_tail(gp[u].astype(np.float64), kk, tail)
+            assert got[u].tolist() == own.tolist(), (n, kk, tail, pool, mode)
+    assert P.spk_device_error() == (0, 0)
+
+
+def test_speckv_avg_pool_end_to_end(P):
+    """speckv_compress with average pooling: scores against the oracle, the
+    selection bit-exact on the GPU's own pooled values and tie-tolerant
+    against the oracle's own average-pooled selection."""
+    import torch
+    qb, kb, vb = _random_case(23, 1, 2, 8, 2, 128, 1500, 32, 32)
+    q, k, v = to_bf16_tensor(qb), to_bf16_tensor(kb), to_bf16_tensor(vb)
+    buf = P.pipeline.SpeckvBuffers(q, k, v, 32, 128, with_pooled=True)
+    P.speckv_compress(q, k, v, 32, 128, 5, buffers=buf, pool_mode=P.SPK_POOL_AVG)
+    torch.cuda.synchronize()
+    scores, pooled, idx = buf.scores.cpu().numpy(), buf.pooled.cpu().numpy(), buf.idx.cpu().numpy()
+    kout = bits_of(buf.k_out)
+    for u in range(buf.units):
+        l, h = u // 2, u % 2
+        s, _ = oracle.speckv_unit(qb[0, l, h * 4:(h + 1) * 4], kb[0, l, h], 32, 32)
+        assert_scores_close(scores[u], s, f"scores[{u}]")
+        np.testing.assert_allclose(pooled[u], oracle.avgpool(scores[u].astype(np.float64), 5), rtol=1e-6, atol=0)
+        assert idx[u].tolist() == oracle.topk_with_tail(pooled[u].astype(np.float64), 128, 32).tolist()
+        p = oracle.avgpool(s, 5)
+        assert_indices_match(idx[u], oracle.topk_with_tail(p, 128, 32), p, 128)
+        np.testing.assert_array_equal(kout[0, l, h], kb[0, l, h][idx[u]])
 
 
 def test_kv_compact_broadcast_and_errors(P):

@@ -25,7 +25,7 @@ __all__ = [
     "SpecKVConfig", "SpecPCConfig", "CascadeConfig", "CONFIGS",
     "bf16_round", "bf16_bits", "bf16_decode",
     "tiny_speckv_numpy", "heavy_positions", "speckv_inputs", "specpc_inputs",
-    "specpc_row_weights",
+    "specpc_row_weights", "speckv_unit_numpy", "specpc_layer_numpy",
 ]
 
 
@@ -355,3 +355,22 @@ def speckv_unit_numpy(cfg: SpecKVConfig, seed: int, unit: int):
     q += cfg.q_offset * u
     q *= np.float32(1.0 / math.sqrt(d))
     return bf16_bits(q), bf16_bits(k), bf16_bits(v)
+
+
+def specpc_layer_numpy(cfg: SpecPCConfig, seed: int, b: int, layer: int):
+    """One (batch element, layer) of a SpecPC draft drawn on the host with
+    numpy: q [Hq, W, d], k [Hkv, n_in, d] (bf16 bit patterns), with the
+    distribution of specpc_inputs (heavy keys of the batch element, one u_h
+    per KV head, query offset; its own random stream)."""
+    rng = np.random.default_rng([seed, b, layer])
+    d = cfg.head_dim
+    q = rng.standard_normal((cfg.hq, cfg.n_rows, d)).astype(np.float32)
+    k = rng.standard_normal((cfg.hkv, cfg.n_in, d)).astype(np.float32)
+    u = _unit(rng.standard_normal((cfg.hkv, d))).astype(np.float32)
+    hp = heavy_positions(cfg.n_in, cfg.heavy_frac, 0, 32, seed * 1000 + b)
+    if cfg.sink:
+        k[:, 0] += cfg.sink * u
+    k[:, hp] += cfg.heavy * u[:, None, :]
+    q += cfg.q_offset * np.repeat(u, cfg.g, axis=0)[:, None, :]
+    q *= np.float32(1.0 / math.sqrt(d))
+    return bf16_bits(q), bf16_bits(k)
