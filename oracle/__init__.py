@@ -54,9 +54,10 @@ def _load():
         lib.oracle_topk_with_tail.argtypes = [_dp, I, I, I, _i32p]
         lib.oracle_gather_rows.argtypes = [_u8p, I, I, _i32p, I, _u8p]
         lib.oracle_decode_row.argtypes = [_u16p, _u16p, _u16p, I, I, D, _dp]
+        lib.oracle_prefill_row.argtypes = [_u16p, _u16p, _u16p, I, I, I, D, _dp, _dp]
         for f in (lib.oracle_speckv_unit, lib.oracle_speckv_unit_f64, lib.oracle_specpc_batch,
                   lib.oracle_specpc_batch_f64, lib.oracle_maxpool, lib.oracle_avgpool, lib.oracle_topk_with_tail,
-                  lib.oracle_gather_rows, lib.oracle_decode_row):
+                  lib.oracle_gather_rows, lib.oracle_decode_row, lib.oracle_prefill_row):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -190,6 +191,35 @@ def decode_attention(q, k, v, scale: float = 1.0):
                                              _ptr(v[b, l, qh // g], _u16p), n_kv, d, scale, _ptr(row, _dp)))
                 out[b, l, qh] = row
     return out
+
+
+def prefill_unit(q, k, v, n_window: int, n_lookahead: int, n_in: int, scale: float = 1.0):
+    """Prefill attention of one unit's window and lookahead rows.
+
+    q [g, R, d] (R = n_window + n_lookahead), k/v [n_in + n_lookahead, d]
+    (input tokens, then the lookahead tokens) as bf16 bit patterns.  Window
+    row i sits at position n_in - n_window + i, lookahead row i at
+    n_in + (i - n_window); each attends to the keys up to its position.
+    Returns (out [g, R, d] float64, lse_in [g * R], natural log over the
+    input keys only)."""
+    lib = _load()
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    g, R, d = q.shape
+    assert R == n_window + n_lookahead and k.shape == v.shape and k.shape[0] >= n_in + n_lookahead
+    out = np.zeros((g, R, d), np.float64)
+    lse = np.zeros(g * R, np.float64)
+    for h in range(g):
+        for i in range(R):
+            pos = n_in - n_window + i if i < n_window else n_in + (i - n_window)
+            row = np.zeros(d, np.float64)
+            l = ctypes.c_double(0.0)
+            _check(lib.oracle_prefill_row(_ptr(q[h, i], _u16p), _ptr(k, _u16p), _ptr(v, _u16p), pos + 1, n_in, d,
+                                          scale, _ptr(row, _dp), ctypes.byref(l)))
+            out[h, i] = row
+            lse[h * R + i] = l.value
+    return out, lse
 
 
 def speckv_select_unit(q, k, n_window, n_lookahead, c_max, pool=7, scale=1.0):

@@ -308,3 +308,51 @@ int oracle_decode_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, i
     free(z);
     return 0;
 }
+
+/*
+ * Prefill attention of one query row ("Draft-based Approximate Inference for
+ * LLMs", paper notes, section 关键设计, SpecKV: the input tokens and the
+ * lookahead tokens go through the target model's prefill together; the
+ * importance is read from the attention of the last n_window input rows and
+ * the lookahead rows).  The key/value sequence holds the n_in input tokens
+ * followed by the lookahead tokens; the row attends causally to its first c
+ * keys:
+ *   z_j = scale <q, k_j>  (j < c),   p = softmax(z),   out = sum_j p_j v_j,
+ *   lse_in = log sum_{j < min(c, n_in)} exp(z_j)   (over the INPUT keys only:
+ *            the normaliser the importance scores use).
+ * q [d], k [c][d], v [c][d] as bf16 bit patterns (rows >= c are not read);
+ * out [d] and *lse_in in double.
+ */
+int oracle_prefill_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, int c, int n_in, int d,
+                       double scale, double *out, double *lse_in) {
+    if (c < 1 || n_in < 1 || d < 1) return -1;
+    double *z = (double *)malloc((size_t)c * sizeof(double));
+    if (!z) return -1;
+    double zmax = -INFINITY;
+    for (int j = 0; j < c; ++j) {
+        double dot = 0.0;
+        for (int t = 0; t < d; ++t) dot += bf16_to_double(q[t]) * bf16_to_double(k[(size_t)j * d + t]);
+        z[j] = scale * dot;
+        if (z[j] > zmax) zmax = z[j];
+    }
+    /* the input keys' log-sum-exp, max-subtracted on its own maximum */
+    const int c_in = c < n_in ? c : n_in;
+    double mi = -INFINITY;
+    for (int j = 0; j < c_in; ++j)
+        if (z[j] > mi) mi = z[j];
+    double si = 0.0;
+    for (int j = 0; j < c_in; ++j) si += exp(z[j] - mi);
+    *lse_in = mi + log(si);
+    double den = 0.0;
+    for (int j = 0; j < c; ++j) {
+        z[j] = exp(z[j] - zmax);
+        den += z[j];
+    }
+    for (int t = 0; t < d; ++t) out[t] = 0.0;
+    for (int j = 0; j < c; ++j) {
+        const double pj = z[j] / den;
+        for (int t = 0; t < d; ++t) out[t] += pj * bf16_to_double(v[(size_t)j * d + t]);
+    }
+    free(z);
+    return 0;
+}
