@@ -134,6 +134,39 @@ spk_status speckv_score_static_ws(const spk_speckv_shape* shape, const void* q_b
                                   float* scores, float* window_mass, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Prefill attention of the window and lookahead rows (section 关键设计,
+ * SpecKV: the input tokens and the lookahead tokens go through the target
+ * model's prefill together, and the importance scores are read from the
+ * attention of the last n_window input rows and of the lookahead rows)
+ *
+ * The key/value sequence of a unit is its n_in input tokens followed by its
+ * n_lookahead lookahead tokens.  Query row i of a head (R = n_window +
+ * n_lookahead rows, ordered as for speckv_score) sits at position
+ * n_in - n_window + i and attends causally to the keys up to that position:
+ *   out[u][row]   = softmax_j(scale * q_row . k_j) . v_j over those keys
+ *   lse2[u][row]  = log2 sum_{j < min(pos + 1, n_in)} 2^(scale*log2(e) * q_row . k_j)
+ *                   -- the same input-key normaliser as speckv_row_lse
+ *   workspace     = (when non-NULL) the row offsets exactly as
+ *                   speckv_row_offsets writes them, so that speckv_colsum on
+ *                   the same shape, q and k gives the importance scores
+ *                   without the scoring's own first pass.
+ *
+ *   q              bf16 [batch][layers][hq][R][head_dim]
+ *   k, v           bf16 [batch][layers][hkv][n_in][head_dim]         (input tokens)
+ *   k_look, v_look bf16 [batch][layers][hkv][n_lookahead][head_dim]  (NULL if n_lookahead = 0)
+ *   out            bf16 [batch][layers][hq][R][head_dim]
+ *   lse2           fp32 [units][g * R] or NULL
+ *   workspace      NULL, or speckv_workspace_size(shape) bytes, 16-byte aligned
+ * Probabilities enter the P.V product as bf16 (fp32 accumulation); the
+ * normaliser and lse2 are formed from the fp32 probabilities.
+ * Supported: as speckv_score.
+ * ------------------------------------------------------------------------ */
+spk_status speckv_prefill_attention(const spk_speckv_shape* shape, const void* q_bf16, const void* k_bf16,
+                                   const void* v_bf16, const void* k_look_bf16, const void* v_look_bf16,
+                                   void* out_bf16, float* lse2, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/* ------------------------------------------------------------------------
  * SpecPC scoring (section 关键设计, SpecPC)
  *
  * Per batch element b, the draft's last W = n_rows query positions: row i sits
@@ -201,9 +234,8 @@ spk_status specpc_colsum(const spk_specpc_shape* shape, const void* q_bf16, cons
  *
  * The pages say "local pooling" without its kind; the workloads use max
  * pooling, which is what topk_select does.  topk_select_pool takes the mode.
- * The workspace is used only when k > 2048 or more than 2048 pooled values
- * fall into the 12-bit key bin of the k-th largest (long runs of equal
- * values); it must always be given.
+ * Workspace: units * round_up(n_cand, 4) * 4 bytes, 16-byte aligned (the
+ * order-preserving 32-bit keys of the pooled values, one padded row per unit).
  *
  * Supported: pool_kernel odd >= 1; k >= 0; n_tail >= 0; n_cand >= 0;
  * pool_mode SPK_POOL_MAX or SPK_POOL_AVG.

@@ -17,7 +17,7 @@ from __future__ import annotations
 from .binding import (  # noqa: F401
     SpeckvError, load_library, library_path,
     speckv_workspace_size, speckv_score, speckv_row_lse, speckv_row_offsets, speckv_colsum,
-    specpc_workspace_size, specpc_score, specpc_row_offsets, specpc_colsum,
+    speckv_prefill_attention, specpc_workspace_size, specpc_score, specpc_row_offsets, specpc_colsum,
     topk_workspace_size, topk_select, kv_compact, decode_attention,
     spk_device_error, spk_selftest_wait_timeout, spk_exp2_fma, mapped_host_pointer,
     SPK_POOL_MAX, SPK_POOL_AVG,
@@ -27,7 +27,7 @@ from .pipeline import speckv_compress, specpc_select, cascade_compress  # noqa: 
 __all__ = [
     "SpeckvError", "load_library", "library_path",
     "speckv_workspace_size", "speckv_score", "speckv_row_lse", "speckv_row_offsets", "speckv_colsum",
-    "specpc_workspace_size", "specpc_score", "specpc_row_offsets", "specpc_colsum",
+    "speckv_prefill_attention", "specpc_workspace_size", "specpc_score", "specpc_row_offsets", "specpc_colsum",
     "topk_workspace_size", "topk_select", "kv_compact", "decode_attention",
     "spk_device_error", "spk_selftest_wait_timeout", "spk_exp2_fma", "mapped_host_pointer",
     "SPK_POOL_MAX", "SPK_POOL_AVG", "speckv_compress", "specpc_select", "cascade_compress",

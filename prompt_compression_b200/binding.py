@@ -65,6 +65,7 @@ def load_library():
         "speckv_row_lse": (I, [sk, vp, vp, vp, vp]),
         "speckv_row_offsets": (I, [sk, vp, vp, vp, sz, vp]),
         "speckv_colsum": (I, [sk, vp, vp, vp, vp, vp, sz, vp]),
+        "speckv_prefill_attention": (I, [sk, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "specpc_workspace_size": (sz, [sp]),
         "specpc_score": (I, [sp, vp, vp, vp, vp, vp, sz, vp]),
         "specpc_row_offsets": (I, [sp, vp, vp, vp, vp, sz, vp]),
@@ -223,6 +224,39 @@ def speckv_colsum(q, k, n_window: int, scores, workspace, window_mass=None, scal
                              _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                              _stream(stream)))
     return scores
+
+
+def speckv_prefill_attention(q, k, v, k_look, v_look, n_window: int, out=None, lse2=None, workspace=None,
+                             scale: float = 1.0, stream=None):
+    """Prefill attention of the window and lookahead rows: q [B, L, Hq, R, d];
+    k, v [B, L, Hkv, n_in, d] (input tokens); k_look, v_look [B, L, Hkv,
+    n_lookahead, d] or None.  Returns out bf16 [B, L, Hq, R, d]; fills lse2
+    (fp32 [units, g*R]) and the column pass's workspace when given."""
+    lib = load_library()
+    shape = speckv_shape(q, k, n_window, scale)
+    units = shape.batch * shape.layers * shape.hkv
+    rows = shape.hq // shape.hkv * (shape.n_window + shape.n_lookahead)
+    if tuple(v.shape) != tuple(k.shape):
+        raise ValueError("v must have k's shape")
+    look = (shape.batch, shape.layers, shape.hkv, shape.n_lookahead, shape.head_dim)
+    if shape.n_lookahead > 0:
+        if k_look is None or v_look is None or tuple(k_look.shape) != look or tuple(v_look.shape) != look:
+            raise ValueError(f"k_look and v_look must be {list(look)}")
+    else:
+        k_look = v_look = None
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    _numel(out, "out", q.numel())
+    _numel(lse2, "lse2", units * rows, required=False)
+    ws_bytes = 0
+    if workspace is not None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.speckv_prefill_attention(ctypes.byref(shape), _dev(q, "q", torch.bfloat16),
+                                        _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+                                        _dev(k_look, "k_look", torch.bfloat16), _dev(v_look, "v_look", torch.bfloat16),
+                                        _dev(out, "out", torch.bfloat16), _dev(lse2, "lse2", torch.float32),
+                                        _dev(workspace, "workspace"), ws_bytes, _stream(stream)))
+    return out
 
 
 def speckv_row_lse(q, k, n_window: int, lse2, scale: float = 1.0, stream=None):

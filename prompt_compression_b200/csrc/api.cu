@@ -122,6 +122,7 @@ ScoreParams base_params(int head_dim, int n_in, const SpeckvGeom& g, int c0, flo
   p.n_in = n_in;
   p.rows = static_cast<int>(g.rows);
   p.R = g.R;
+  p.R_mul = g.R > 1 ? static_cast<uint32_t>(((1ull << 32) + g.R - 1) / g.R) : 0u;
   p.c0 = c0;
   p.c2 = scale * 1.4426950408889634f;
   p.hkv = hkv;
@@ -253,6 +254,59 @@ spk_status speckv_score(const spk_speckv_shape* s, const void* q, const void* k,
   if ((window_mass ? s->n_in : g.n_pre) == 0) return ok();
   if ((st = speckv_row_offsets(s, q, k, ws, ws_bytes, stream)) != SPK_OK) return st;
   return speckv_colsum(s, q, k, scores, window_mass, ws, ws_bytes, stream);
+}
+
+// Prefill attention of the window and lookahead rows (attn.cu): outputs, the
+// input-key LSE and, when a workspace is given, the column pass's row offsets.
+spk_status speckv_prefill_attention(const spk_speckv_shape* s, const void* q, const void* k, const void* v,
+                                   const void* k_look, const void* v_look, void* out, float* lse2, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  SpeckvGeom g;
+  spk_status st = check_speckv(s, g);
+  if (st != SPK_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr)
+    return fail(SPK_ERR_ARG, "q, k, v and out must be non-NULL device pointers");
+  if (s->n_lookahead > 0 && (k_look == nullptr || v_look == nullptr))
+    return fail(SPK_ERR_ARG, "k_look and v_look must be non-NULL when n_lookahead > 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (s->n_lookahead > 0 && (!aligned16(k_look) || !aligned16(v_look))))
+    return fail(SPK_ERR_ARG, "q, k, v, k_look, v_look and out must be 16-byte aligned");
+  if (ws != nullptr) {
+    const size_t need = speckv_workspace_size(s);
+    if (ws_bytes < need) return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
+  }
+  const long long tiles = row_tiles(g.rows);
+  if (g.units * tiles > 0x7fffffffLL) return fail(SPK_ERR_UNSUPPORTED, "too many units");
+  CUtensorMap maps[5];
+  if ((st = make_map(&maps[0], q, s->head_dim, g.rows, g.units)) != SPK_OK) return st;
+  if ((st = make_map(&maps[1], k, s->head_dim, s->n_in, g.units)) != SPK_OK) return st;
+  if ((st = make_map(&maps[2], v, s->head_dim, s->n_in, g.units)) != SPK_OK) return st;
+  if (s->n_lookahead > 0) {
+    if ((st = make_map(&maps[3], k_look, s->head_dim, s->n_lookahead, g.units)) != SPK_OK) return st;
+    if ((st = make_map(&maps[4], v_look, s->head_dim, s->n_lookahead, g.units)) != SPK_OK) return st;
+  } else {
+    maps[3] = maps[1];   // never read: no lookahead tiles
+    maps[4] = maps[2];
+  }
+  AttnParams p;
+  memset(&p, 0, sizeof p);
+  p.head_dim = s->head_dim;
+  p.n_in = s->n_in;
+  p.n_look = s->n_lookahead;
+  p.rows = static_cast<int>(g.rows);
+  p.R = g.R;
+  p.c0 = s->n_in - s->n_window + 1;
+  p.c2 = s->scale * 1.4426950408889634f;
+  p.row_tiles = static_cast<int>(tiles);
+  p.n_items = static_cast<int>(g.units * tiles);
+  p.out = out;
+  p.lse2 = lse2;
+  p.off_blocks = static_cast<uint8_t*>(ws);
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  cudaError_t e = launch_attn(s->head_dim, maps, p, grid, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
+  return ok();
 }
 
 // ------------------------------------------------------------------ SpecPC
@@ -416,6 +470,7 @@ static spk_status topk_common(const float* scores, int units, int n_cand, int po
   const size_t need = topk_workspace_size(units, n_cand);
   if (need > 0 && (ws == nullptr || ws_bytes < need))
     return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+  if (need > 0 && !aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
   if (static_cast<long long>(units) > 0x7fffffffLL / (out_len > 0 ? out_len : 1) && out_len > 0)
     return fail(SPK_ERR_UNSUPPORTED, "output too large");
   cudaError_t e = launch_topk(scores, units, n_cand, pool_mode, pool_kernel, k, n_tail, idx, pooled, ws,

@@ -1,0 +1,444 @@
+// attn.cu -- prefill attention of the window and lookahead rows on tcgen05,
+// emitting the rows' outputs and their input-key log-sum-exp.
+//
+// "Draft-based Approximate Inference for LLMs" (paper notes), section 关键设计,
+// SpecKV: the input tokens and the lookahead tokens go through the target
+// model's prefill together, and the importance of the input KV pairs is read
+// from the attention of the last n_window input rows and the lookahead rows.
+// This kernel is that attention for those rows: row i (head-local) sits at
+// position n_in - n_window + i and attends causally to the keys up to it --
+// the n_in input keys, then (lookahead rows only) the lookahead keys up to
+// its own.  Outputs per row:
+//   out   = softmax(scale q.k) V over the visible keys (bf16)
+//   lse2  = log2 sum_{visible input keys} 2^(c2 q.k), c2 = scale log2(e):
+//           the normaliser of the importance scores, written as the row
+//           offsets the column pass (speckv_colsum) reads, so that scoring
+//           after this attention needs only the column pass.
+//
+// Work decomposition: an item is one unit's 128-row Q tile; a persistent CTA
+// walks items.  Key tiles of 128: phase A over the input keys (tile t at key
+// 128 t; the unit's input K/V tensor map ends at n_in, so the last tile's
+// tail reads as zeros and is masked), then phase B over the lookahead keys
+// (their own tensor map).  After phase A every row's (max, sum) gives the
+// input-key LSE.
+//   warps 0-3 : softmax; thread = query row (TMEM lane).  Per key tile: load
+//               S (128 fp32 columns), row max, lazy rescale (the running max
+//               moves only when a tile's max exceeds it by more than 8 in
+//               log2 units; O and the sum are rescaled then, after the
+//               previous P.V has finished), P = 2^(c2 s - m) into TMEM as
+//               bf16 pairs over the first 64 columns of the S buffer.
+//   warp 4    : TMA producer (Q per item; K and V tiles through a 2-stage ring).
+//   warp 5    : TMEM allocator + single-thread UMMA issuer:
+//               S(t) = Q K(t)^T (A and B from shared memory), then
+//               O += P(t) V(t) (A = P from TMEM, B = V from shared memory in
+//               its natural [key][d] layout, i.e. MN-major).
+// TMEM: S buffers at columns 0 and 128 (P aliases their first 64 columns),
+// O at 256 (head_dim columns).  No atomics: the result is deterministic.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "score.cuh"
+
+namespace spk {
+namespace {
+
+constexpr int kAttnSoftmaxWarps = 4;
+constexpr int kAttnProducerWarp = 4;
+constexpr int kAttnMmaWarp = 5;
+constexpr int kAttnThreads = 6 * 32;
+constexpr float kRescaleLog2 = 8.f;    // lazy rescale threshold (P <= 2^8)
+
+template <int D>
+struct AttnCfg {
+  static constexpr int kTileBytes = 128 * D * 2;   // 128 rows x D bf16 (Q, K or V tile)
+  static constexpr int kAtoms = D / 64;            // 128-byte swizzle atoms along D
+  static constexpr int kStages = 2;
+  static constexpr int kSmemBytes = 1024 + kTileBytes + 2 * kStages * kTileBytes;
+  static_assert(kSmemBytes <= 227 * 1024 - 2048, "fits one CTA");
+};
+
+// Shared-memory descriptor of an MN-major operand in the 128-byte-swizzled
+// layout TMA writes: 128-byte rows along K (here: keys), N (here: head_dim)
+// contiguous inside a row, 8-row (1024-byte) swizzle atoms stacked along K
+// (stride byte offset), 64-element column blocks `lbo` bytes apart along N.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return a | (b << 16);
+}
+
+// Row r (0..127) of a row-offset block: v split into three bf16 terms
+// (the layout the column pass reads; see kOffBlockBytes).
+__device__ __forceinline__ void attn_store_offset_row(uint8_t* block, int r, float v) {
+  const __nv_bfloat16 h1 = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h1);
+  const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(h2);
+  const __nv_bfloat16 h3 = __float2bfloat16_rn(r2);
+  const uint32_t w0 = static_cast<uint32_t>(__bfloat16_as_ushort(h1)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(h2)) << 16);
+  const uint32_t w1 = static_cast<uint32_t>(__bfloat16_as_ushort(h3));
+  uint8_t* row = block + (r >> 3) * 256 + (r & 7) * 16;
+  *reinterpret_cast<uint4*>(row) = make_uint4(w0, w1, 0u, 0u);
+  *reinterpret_cast<uint4*>(row + 128) = make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ int attn_site(int role, int which) { return 300 + role * 10 + which; }
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap klmap,
+                const __grid_constant__ CUtensorMap vlmap, const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* const Q_s = smem;
+  uint8_t* const K_s = smem + C::kTileBytes;
+  uint8_t* const V_s = K_s + C::kStages * C::kTileBytes;
+
+  __shared__ __align__(8) uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
+      p_full[2], pv_done, o_empty, done_bar;
+  __shared__ uint32_t tmem_holder;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tiles_a = (p.n_in + 127) / 128;
+  const int tiles_b = (p.n_look + 127) / 128;
+  const int n_tiles = tiles_a + tiles_b;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kAttnSoftmaxWarps);
+    }
+    mbar_init(&pv_done, 1);
+    mbar_init(&o_empty, kAttnSoftmaxWarps);
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kAttnMmaWarp) {
+    tmem_alloc(&tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == kAttnProducerWarp && lane == 0) {
+    tma_prefetch_map(&qmap);
+    tma_prefetch_map(&kmap);
+    tma_prefetch_map(&vmap);
+    if (tiles_b > 0) {
+      tma_prefetch_map(&klmap);
+      tma_prefetch_map(&vlmap);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+  volatile int* abort_v = &abort_flag;
+
+  if (warp == kAttnProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t tile_count = 0;     // K/V tiles loaded by this CTA (stage = count % 2)
+      int items_done = 0;
+      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1}, q_last = -1;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
+        const int u = item / p.row_tiles, rb = item % p.row_tiles;
+        if (!(ok = mbar_wait(&q_empty, (items_done & 1) ^ 1, abort_v, attn_site(0, 0)))) break;
+        mbar_arrive_expect_tx(&q_full, C::kTileBytes);
+        for (int a = 0; a < C::kAtoms; ++a) tma_load_3d(Q_s + a * 16384, &qmap, &q_full, a * 64, rb * 128, u);
+        q_last = items_done & 1;
+        for (int t = 0; ok && t < n_tiles; ++t, ++tile_count) {
+          const int st = tile_count & 1;
+          const uint32_t ph = (tile_count >> 1) & 1;
+          const bool in_a = t < tiles_a;
+          const int row0 = in_a ? t * 128 : (t - tiles_a) * 128;
+          if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, abort_v, attn_site(0, 1)))) break;
+          mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+          for (int a = 0; a < C::kAtoms; ++a)
+            tma_load_3d(K_s + st * C::kTileBytes + a * 16384, in_a ? &kmap : &klmap, &k_full[st], a * 64, row0, u);
+          k_last[st] = static_cast<int>(ph);
+          if (!(ok = mbar_wait(&v_empty[st], ph ^ 1, abort_v, attn_site(0, 2)))) break;
+          mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
+          for (int a = 0; a < C::kAtoms; ++a)
+            tma_load_3d(V_s + st * C::kTileBytes + a * 16384, in_a ? &vmap : &vlmap, &v_full[st], a * 64, row0, u);
+          v_last[st] = static_cast<int>(ph);
+        }
+      }
+      if (!ok) {
+        volatile int never = 0;
+        if (q_last >= 0) mbar_wait(&q_full, q_last, &never, attn_site(0, 7), 100000000ull);
+        for (int s = 0; s < 2; ++s) {
+          if (k_last[s] >= 0) mbar_wait(&k_full[s], k_last[s], &never, attn_site(0, 8), 100000000ull);
+          if (v_last[s] >= 0) mbar_wait(&v_full[s], v_last[s], &never, attn_site(0, 9), 100000000ull);
+        }
+      }
+    }
+  } else if (warp == kAttnMmaWarp) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t T = 0;              // key tiles of this CTA before the current item
+      int items_done = 0;
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 64) | (1u << 16);   // B (V) MN-major
+      const uint64_t q_desc = sw128_kmajor_desc(smem_u32(Q_s));
+      auto issue_s = [&](uint32_t Ti) -> bool {
+        const int st = Ti & 1;
+        if (!mbar_wait(&k_full[st], (Ti >> 1) & 1, abort_v, attn_site(1, 1))) return false;
+        tc_fence_after();
+        const uint64_t k_desc = sw128_kmajor_desc(smem_u32(K_s + st * C::kTileBytes));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_bf16_ss(tmem_base + st * 128, q_desc + koff, k_desc + koff, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[st]);
+        umma_commit(&k_empty[st]);
+        return true;
+      };
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
+        if (!(ok = mbar_wait(&q_full, items_done & 1, abort_v, attn_site(1, 0)))) break;
+        // S(0) overwrites the buffer P(T - 2) used.  Wait for the previous
+        // item's last P.V (it implies the earlier ones): a parity wait is only
+        // unambiguous for the newest phase or the one before it.
+        if (T >= 1 && !(ok = mbar_wait(&pv_done, (T - 1) & 1, abort_v, attn_site(1, 2)))) break;
+        if (!(ok = issue_s(T))) break;
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const uint32_t Tc = T + t;
+          if (t + 1 < n_tiles) {
+            // buffer (Tc + 1) % 2 held P(Tc - 1): wait for its P.V
+            if (Tc >= 1 && !(ok = mbar_wait(&pv_done, (Tc - 1) & 1, abort_v, attn_site(1, 3)))) break;
+            if (!(ok = issue_s(Tc + 1))) break;
+          }
+          const int st = Tc & 1;
+          if (!(ok = mbar_wait(&p_full[st], (Tc >> 1) & 1, abort_v, attn_site(1, 4)))) break;
+          if (!(ok = mbar_wait(&v_full[st], (Tc >> 1) & 1, abort_v, attn_site(1, 5)))) break;
+          // the softmax warps have read the previous item's O before it is restarted
+          if (t == 0 && items_done > 0 && !(ok = mbar_wait(&o_empty, (items_done - 1) & 1, abort_v, attn_site(1, 6))))
+            break;
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(V_s + st * C::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int a = 0; a < C::kAtoms; ++a) {
+              const uint64_t v_desc = sw128_mnmajor_desc(v_base + a * 16384 + kk * 2048, 16384);
+              umma_bf16_ts(tmem_base + 256 + a * 64, tmem_base + st * 128 + kk * 8, v_desc, idesc_pv,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&v_empty[st]);
+          umma_commit(&pv_done);
+        }
+        if (!ok) break;
+        umma_commit(&q_empty);
+        T += n_tiles;
+      }
+      umma_commit(&done_bar);
+      volatile int never = 0;
+      mbar_wait(&done_bar, 0, &never, attn_site(1, 9), 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int r = warp * 32 + lane;                     // row within the Q tile = TMEM lane
+    const uint32_t tlane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    bool ok = true;
+    uint32_t T = 0;
+    int items_done = 0;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, int which) -> bool {
+      bool w = mbar_wait(bar, parity, abort_v, attn_site(2, which));
+      return __all_sync(0xffffffffu, w);
+    };
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
+      const int u = item / p.row_tiles, rb = item % p.row_tiles;
+      const int n = rb * 128 + r;                       // row within the unit
+      const bool live = n < p.rows;
+      const int c = p.c0 + n % p.R;                     // visible keys (input, then lookahead)
+      float m = -INFINITY, l = 0.f, lse_in = 0.f;       // m: running max of c2 * s
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        const uint32_t Tc = T + t;
+        const int buf = Tc & 1;
+        if (!(ok = wait_all(&s_full[buf], (Tc >> 1) & 1, 0))) break;
+        tc_fence_after();
+        // keys of this tile this row sees: [0, lim)
+        const bool in_a = t < tiles_a;
+        const int j0 = in_a ? t * 128 : p.n_in + (t - tiles_a) * 128;
+        const int j_end = in_a ? min(j0 + 128, p.n_in) : min(j0 + 128, p.n_in + p.n_look);
+        const int lim = max(0, min(c, j_end) - j0);
+        float s[128];
+        {
+          uint32_t a0[32], a1[32];
+          tmem_ld32(tlane + buf * 128, a0);
+          tmem_ld32(tlane + buf * 128 + 32, a1);
+          tmem_ld_wait2(a0, a1);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) { s[k] = __uint_as_float(a0[k]); s[32 + k] = __uint_as_float(a1[k]); }
+          tmem_ld32(tlane + buf * 128 + 64, a0);
+          tmem_ld32(tlane + buf * 128 + 96, a1);
+          tmem_ld_wait2(a0, a1);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) { s[64 + k] = __uint_as_float(a0[k]); s[96 + k] = __uint_as_float(a1[k]); }
+        }
+        if (lim < 128) {
+#pragma unroll
+          for (int k = 0; k < 128; ++k)
+            if (k >= lim) s[k] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 128; k += 4) mx = fmaxf(mx, max3f(s[k], s[k + 1], fmaxf(s[k + 2], s[k + 3])));
+        const float mt = mx * p.c2;
+        const bool need = lim > 0 && mt > m + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m - mt) : 1.f;   // m = -inf: alpha = 0
+          if (t > 0) {
+            // O holds the P.V products of tiles 0 .. t-1: rescale it once the last has landed
+            if (!(ok = wait_all(&pv_done, (Tc - 1) & 1, 1))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t o[32];
+              tmem_ld32(tlane + 256 + ch * 32, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32(tlane + 256 + ch * 32, o);
+            }
+            tmem_st_wait();
+          }
+          if (need) {
+            l *= alpha;
+            m = mt;
+          }
+        }
+        // P = 2^(c2 s - m) (masked keys: 2^-inf = 0), packed as bf16 pairs
+        float sum0 = 0.f, sum1 = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          const float e0 = ex2_approx(fmaf(s[2 * k], p.c2, -m));
+          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.c2, -m));
+          sum0 += e0;
+          sum1 += e1;
+          pk[k] = pack_bf16(e0, e1);
+        }
+        l += sum0 + sum1;
+        {
+          uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+          uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+          tmem_st32(tlane + buf * 128, p0);
+          tmem_st32(tlane + buf * 128 + 32, p1);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[buf]);
+        if (t == tiles_a - 1) lse_in = m + lg2_approx(l);   // every input key is in
+      }
+      if (!ok) break;
+      // ---- O of this item: after the last P.V, scale by 1 / l and store
+      // P.V(Tl - 2) has finished (S(Tl) was issued after it), so the phases
+      // of P.V(Tl - 1) and then P.V(Tl) are the two newest: wait for both
+      const uint32_t Tl = T + n_tiles - 1;
+      if (Tl >= 1 && !(ok = wait_all(&pv_done, (Tl - 1) & 1, 2))) break;
+      if (!(ok = wait_all(&pv_done, Tl & 1, 3))) break;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                            (static_cast<size_t>(u) * p.rows + (live ? n : 0)) * D;
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tlane + 256 + ch * 32, o);
+        tmem_ld_wait(o);
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+            w.y = pack_bf16(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+            w.z = pack_bf16(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+            w.w = pack_bf16(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+            dst[v4] = w;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty);
+      if (p.lse2 != nullptr && live) p.lse2[static_cast<size_t>(u) * p.rows + n] = lse_in;
+      if (p.off_blocks != nullptr)
+        attn_store_offset_row(p.off_blocks + (static_cast<size_t>(u) * p.row_tiles + rb) * kOffBlockBytes, r,
+                              live ? -lse_in / p.c2 : -1e30f);
+      T += n_tiles;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kAttnMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int D>
+static cudaError_t attn_launch_one(const CUtensorMap (&maps)[5], const AttnParams& p, int grid,
+                                   cudaStream_t stream) {
+  using C = AttnCfg<D>;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  attn_kernel<D><<<grid, kAttnThreads, C::kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn(int head_dim, const CUtensorMap (&maps)[5], const AttnParams& p, int grid,
+                        cudaStream_t stream) {
+  if (head_dim == 128) return attn_launch_one<128>(maps, p, grid, stream);
+  if (head_dim == 64) return attn_launch_one<64>(maps, p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace spk

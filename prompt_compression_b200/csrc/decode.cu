@@ -9,17 +9,19 @@
 // over the n_kv rows of the head's KV head (GQA: query head qh reads KV head
 // qh / g), e.g. the k_out / v_out that kv_compact leaves.
 //
-// One CTA (8 warps) per (batch, layer, KV head) unit; warp w takes the
-// 32-row blocks w, w + 8, ...  Within a block, lane l owns row t0 + l for the
-// logits: it reads its K row in 16-byte pieces and dots it with the g query
-// rows held in shared memory (broadcast reads), so no cross-lane reduction
-// is needed per row.  The block's max and sum per query head take one warp
-// reduction each (online softmax: log2-domain running max and sum), the
-// weights go to shared memory, and for the weighted V sum lane l owns
-// elements [l * d/32, (l + 1) * d/32) of every V row (coalesced row loads).
-// At the end the 8 warps' states are merged in a fixed order, so results
-// are bitwise reproducible.  Every K and V byte is read once: the kernel is
-// bound by HBM bandwidth.
+// One CTA per (batch, layer, KV head) unit, one warp per 32-row block (up to
+// 16 warps; with more blocks each warp takes blocks w, w + warps, ...).  For
+// its block a warp first issues the copy of the 32 V rows into its own
+// shared-memory buffer (cp.async, 16 bytes per lane per copy), then reads
+// the K rows: lane l owns row t0 + l, requests the whole row at once and
+// dots it with the g query rows held in shared memory (broadcast reads), so
+// no cross-lane reduction is needed per row.  K and V of the block are thus
+// in flight together.  The block's max and sum per query head take one warp
+// reduction each (online softmax: log2-domain running max and sum); for the
+// weighted V sum lane l owns elements [l * d/32, (l + 1) * d/32) of every V
+// row, read from shared memory.  At the end the warps' states are merged in
+// a fixed order, so results are bitwise reproducible.  Every K and V byte is
+// read once: the kernel is bound by HBM bandwidth.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -28,7 +30,13 @@
 namespace spk {
 namespace {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecMaxWarps = 16;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 template <int D>
 struct RowSlice;   // one lane's d/32 bf16 elements of a row
@@ -60,19 +68,21 @@ __device__ __forceinline__ void unpack(const typename RowSlice<D>::T& r, float (
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecWarps * 32)
+__global__ void __launch_bounds__(kDecMaxWarps * 32)
     decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
                   float* __restrict__ out, int n_kv, float c2) {
   using S = RowSlice<D>;
-  constexpr int E = S::kN;   // V elements per lane
+  constexpr int E = S::kN;                    // V elements per lane
+  constexpr int kBlockBytes = 32 * D * 2;     // one warp's V block
+  extern __shared__ __align__(16) uint8_t dec_smem[];   // [warps][kBlockBytes]; reused by the merge
   __shared__ __align__(16) float q_s[G][D];
-  __shared__ float p_s[kDecWarps][G][32];
-  __shared__ float m_s[kDecWarps][G], l_s[kDecWarps][G];
-  __shared__ float acc_s[kDecWarps][G][D];
+  __shared__ float p_s[kDecMaxWarps][G][32];
+  __shared__ float m_s[kDecMaxWarps][G], l_s[kDecMaxWarps][G];
 
   const int unit = blockIdx.x;   // (b * layers + l) * hkv + h; its query heads are rows unit*G .. unit*G+G-1
+  const int warps = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < G * D; i += kDecWarps * 32)
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x)
     q_s[i / D][i % D] = __uint_as_float(static_cast<uint32_t>(q[static_cast<size_t>(unit) * G * D + i]) << 16);
   __syncthreads();
 
@@ -85,9 +95,18 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
   }
   const uint16_t* kr = k + static_cast<size_t>(unit) * n_kv * D;
-  const typename S::T* vr = reinterpret_cast<const typename S::T*>(v + static_cast<size_t>(unit) * n_kv * D);
+  const uint8_t* vbytes = reinterpret_cast<const uint8_t*>(v + static_cast<size_t>(unit) * n_kv * D);
+  uint8_t* vbuf = dec_smem + warp * kBlockBytes;
 
-  for (int t0 = warp * 32; t0 < n_kv; t0 += kDecWarps * 32) {
+  for (int t0 = warp * 32; t0 < n_kv; t0 += warps * 32) {
+    const int rows = n_kv - t0 < 32 ? n_kv - t0 : 32;
+    // the block's V rows -> shared memory, in flight while K is read
+    {
+      const uint8_t* src = vbytes + static_cast<size_t>(t0) * D * 2;
+      const int chunks = rows * (D * 2 / 16);
+      for (int c = lane; c < chunks; c += 32) cp_async16(vbuf + c * 16, src + c * 16);
+      cp_async_commit();
+    }
     const int t = t0 + lane;
     const bool valid = t < n_kv;
     // logits of this lane's row for every query head of the group
@@ -136,13 +155,14 @@ __global__ void __launch_bounds__(kDecWarps * 32)
       for (int e = 0; e < E; ++e) acc[h][e] *= alpha;
       p_s[warp][h][lane] = pz;
     }
+    cp_async_wait_all();
     __syncwarp();
-    // weighted V sum over the block's rows; lane owns E elements of a row
-    const int rows = n_kv - t0 < 32 ? n_kv - t0 : 32;
-#pragma unroll 8
+    // weighted V sum over the block's rows (from shared memory); lane owns E elements of a row
+    const typename S::T* vs = reinterpret_cast<const typename S::T*>(vbuf);
+#pragma unroll 4
     for (int j = 0; j < rows; ++j) {
       float vf[E];
-      unpack<D>(__ldcs(vr + static_cast<size_t>(t0 + j) * 32 + lane), vf);
+      unpack<D>(vs[j * 32 + lane], vf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float pj = p_s[warp][h][j];
@@ -150,9 +170,11 @@ __global__ void __launch_bounds__(kDecWarps * 32)
         for (int e = 0; e < E; ++e) acc[h][e] = fmaf(pj, vf[e], acc[h][e]);
       }
     }
-    __syncwarp();
+    __syncwarp();   // the buffer and p_s are free for the next block
   }
-  // merge the warps' states in a fixed order
+  // merge the warps' states in a fixed order (acc_s reuses the V buffers)
+  __syncthreads();
+  float* acc_s = reinterpret_cast<float*>(dec_smem);   // [warps][G][D]
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     if (lane == 0) {
@@ -160,19 +182,19 @@ __global__ void __launch_bounds__(kDecWarps * 32)
       l_s[warp][h] = l[h];
     }
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc_s[warp][h][lane * E + e] = acc[h][e];
+    for (int e = 0; e < E; ++e) acc_s[(warp * G + h) * D + lane * E + e] = acc[h][e];
   }
   __syncthreads();
-  for (int x = threadIdx.x; x < G * D; x += kDecWarps * 32) {
+  for (int x = threadIdx.x; x < G * D; x += blockDim.x) {
     const int h = x / D, c = x % D;
     float M = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, m_s[w][h]);
+    for (int w = 0; w < warps; ++w) M = fmaxf(M, m_s[w][h]);
     float L = 0.f, A = 0.f;
-    for (int w = 0; w < kDecWarps; ++w) {
+    for (int w = 0; w < warps; ++w) {
       if (m_s[w][h] == -INFINITY) continue;   // a warp that saw no row
       const float f = ex2_approx(m_s[w][h] - M);
       L = fmaf(l_s[w][h], f, L);
-      A = fmaf(acc_s[w][h][c], f, A);
+      A = fmaf(acc_s[(w * G + h) * D + c], f, A);
     }
     out[(static_cast<size_t>(unit) * G + h) * D + c] = A / L;
   }
@@ -181,9 +203,23 @@ __global__ void __launch_bounds__(kDecWarps * 32)
 template <int D, int G>
 cudaError_t launch_g(const void* q, const void* k, const void* v, float* out, int units, int n_kv, float c2,
                      cudaStream_t stream) {
-  decode_kernel<D, G><<<units, kDecWarps * 32, 0, stream>>>(static_cast<const uint16_t*>(q),
-                                                            static_cast<const uint16_t*>(k),
-                                                            static_cast<const uint16_t*>(v), out, n_kv, c2);
+  // one warp per 32-row block, up to 16; each warp's V block in shared memory
+  int warps = (n_kv + 31) / 32;
+  warps = warps < 1 ? 1 : (warps > kDecMaxWarps ? kDecMaxWarps : warps);
+  const int smem = warps * 32 * D * 2;
+  static_assert(32 * D * 2 >= G * D * 4, "a warp's V buffer holds its merge state");
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDecMaxWarps * 32 * D * 2);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  decode_kernel<D, G><<<units, warps * 32, smem, stream>>>(static_cast<const uint16_t*>(q),
+                                                           static_cast<const uint16_t*>(k),
+                                                           static_cast<const uint16_t*>(v), out, n_kv, c2);
   return cudaGetLastError();
 }
 

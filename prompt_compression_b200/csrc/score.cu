@@ -92,6 +92,13 @@ struct Cfg {
   static constexpr uint32_t kNumAcc = kATmem ? 3 : 4;
 };
 
+// n / R and n % R for 0 <= n <= 4096 (rows of a unit, R <= 2048) by a
+// multiply-high with ceil(2^32 / R): n * R < 2^32 keeps the quotient exact.
+__device__ __forceinline__ int div_R(const ScoreParams& p, int n) {
+  return p.R == 1 ? n : static_cast<int>(__umulhi(static_cast<uint32_t>(n), p.R_mul));
+}
+__device__ __forceinline__ int mod_R(const ScoreParams& p, int n) { return n - div_R(p, n) * p.R; }
+
 // Error sites: mode * 100 + role * 10 + barrier.
 __device__ __forceinline__ int site(int mode, int role, int which) { return mode * 100 + role * 10 + which; }
 
@@ -247,9 +254,8 @@ __device__ __forceinline__ float fold(const float2 (&s)[4]) {
 
 // For a key j that some rows cannot see: row n (head-local i = n % R) sees
 // key j only if j < c0 + i.  nb is the first row of the 32.
-__device__ __forceinline__ float colsum32_masked(const uint32_t (&v)[32], int nb, float c2, int j, int c0, int R) {
+__device__ __forceinline__ float colsum32_masked(const uint32_t (&v)[32], int i, float c2, int j, int c0, int R) {
   float s = 0.f;
-  int i = nb % R;
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
     if (j < c0 + i) s += ex2_approx(__uint_as_float(v[k]) * c2);
@@ -548,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (MODE == MODE_LSE) {
           const int row = a_row0 + r;
           const bool row_ok = active && row < p.rows;
-          const int c = min(p.n_in, p.c0 + (row_ok ? row % p.R : 0));
+          const int c = min(p.n_in, p.c0 + (row_ok ? mod_R(p, row) : 0));
           for (int bt = 0; bt < nb; ++bt) {
             if (!(ok = wait_acc(0))) break;
             if (active) {
@@ -578,13 +584,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // 3: the group wraps into the next head (per-row test)
           auto mask_class = [&](int nb0) -> int {
             if (!__any_sync(0xffffffffu, m_lane >= 0)) return 0;
-            const int i0 = nb0 % p.R;
+            const int i0 = mod_R(p, nb0);
             if (i0 + 32 > p.R) return 3;
             if (__reduce_max_sync(0xffffffffu, m_lane) < i0) return 0;
             if (__reduce_min_sync(0xffffffffu, m_lane) >= i0 + 31) return 1;
             return 2;
           };
-          const int gh = p.rows / p.R;           // query heads of the unit
+          const int gh = div_R(p, p.rows);       // query heads of the unit
           const int head0 = (seg / p.layers_used) * gh;   // SpecPC: first query head of this KV head
           float seg_sum = 0.f;
           int cur_head = -1;
@@ -604,15 +610,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (mc == 0) {
                   colsum32<kPolyPairsOf8>(v, p.c2, sacc);
                 } else if (mc == 2) {
-                  colsum32<kPolyPairsOf8, true>(v, p.c2, sacc, min(32, max(0, m_lane - nb0 % p.R + 1)));
+                  colsum32<kPolyPairsOf8, true>(v, p.c2, sacc, min(32, max(0, m_lane - mod_R(p, nb0) + 1)));
                 } else if (mc == 3) {
-                  if (masked_key) acc_masked += colsum32_masked(v, nb0, p.c2, j, p.c0, p.R);
+                  if (masked_key) acc_masked += colsum32_masked(v, mod_R(p, nb0), p.c2, j, p.c0, p.R);
                   else colsum32<kPolyPairsOf8>(v, p.c2, sacc);
                 }
               } else {
                 // SpecPC: rows of one query head are contiguous (R = W rows);
                 // rows >= p.rows are padding and belong to no head
-                const int h0 = nb0 / p.R, h1 = (nb0 + 31) / p.R;
+                const int h0 = div_R(p, nb0), h1 = div_R(p, nb0 + 31);
                 if (h0 >= gh) {
                   // the whole group is padding
                 } else if (h0 == h1) {
@@ -629,16 +635,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     seg_sum += fold(gs);
                   } else if (mc == 2) {
                     float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-                    colsum32<kPolyPairsOf8, true>(v, p.c2, gs, min(32, max(0, m_lane - nb0 % p.R + 1)));
+                    colsum32<kPolyPairsOf8, true>(v, p.c2, gs, min(32, max(0, m_lane - mod_R(p, nb0) + 1)));
                     seg_sum += fold(gs);
                   }
                 } else {
                   // a 32-row group that straddles two query heads
-                  int i = nb0 % p.R;
+                  int i = mod_R(p, nb0);
                   for (int k = 0; k < 32; ++k) {
                     const int n = nb0 + k;
                     if (n >= p.rows) break;
-                    const int hh = n / p.R;
+                    const int hh = div_R(p, n);
                     if (hh != cur_head) {
                       if (cur_head >= 0) my_acc[(head0 + cur_head) * 256 + r] += seg_sum;
                       cur_head = hh;
@@ -692,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // weight w_i folds in as -log2(w_i); a row of weight 0 adds
                 // nothing and takes the padding offset (log2(0) = -inf would
                 // turn the three-term split into NaN)
-                const float w = p.row_weights[row % p.R];
+                const float w = p.row_weights[mod_R(p, row)];
                 if (w > 0.f) out += log2_norm - log2f(w);
                 else live = false;
               }
@@ -728,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           arrive_warp(&mrg_full[0]);
         } else {
           if (!(ok = wait_uniform(&mrg_full[0], items_done & 1, 1))) break;
-          const int hq = (p.rows / p.R) * p.hkv;
+          const int hq = div_R(p, p.rows) * p.hkv;
           const int blk = item / p.seg_groups;
           if (p.seg_groups == 1) {
             float best = -INFINITY;

@@ -33,6 +33,7 @@ struct ScoreParams {
   int n_in;          // input keys per unit
   int rows;          // query rows per unit = g * R, ordered [query head][row]
   int R;             // rows per query head
+  uint32_t R_mul;    // ceil(2^32 / R) for R > 1: n / R = umulhi(n, R_mul), exact while n * R < 2^32
   int c0;            // head-local row i sees keys [0, min(n_in, c0 + i))
   float c2;          // scale * log2(e)
   // unit u = (b * layers_used + l') * hkv + h  ->  tensor coordinate
@@ -72,6 +73,26 @@ cudaError_t launch_score(int mode, int head_dim, const CUtensorMap& amap, const 
 cudaError_t launch_specpc_merge(const float* part, int batch, int n_in, int n_blocks, int groups, int hq,
                                 float* scores, cudaStream_t stream);
 int score_smem_bytes(int mode, int head_dim);
+
+// prefill attention of the window and lookahead rows (attn.cu)
+struct AttnParams {
+  int head_dim;
+  int n_in;          // input keys per unit
+  int n_look;        // lookahead keys per unit
+  int rows;          // query rows per unit = g * R, ordered [query head][row]
+  int R;             // rows per query head
+  uint32_t R_mul;    // ceil(2^32 / R) for R > 1: n / R = umulhi(n, R_mul), exact while n * R < 2^32
+  int c0;            // head-local row i sees keys [0, c0 + i) of input + lookahead
+  float c2;          // scale * log2(e)
+  int row_tiles;     // 128-row Q tiles per unit
+  int n_items;       // units * row_tiles
+  void* out;         // bf16 [units][rows][head_dim]
+  float* lse2;       // fp32 [units][rows] or null: log2-domain LSE over the input keys
+  uint8_t* off_blocks;   // row offsets for the column pass (row_tiles blocks per unit) or null
+};
+// maps: q [units][rows][d], k and v [units][n_in][d], lookahead k and v [units][n_look][d]
+cudaError_t launch_attn(int head_dim, const CUtensorMap (&maps)[5], const AttnParams& p, int grid,
+                        cudaStream_t stream);
 
 // pooling + top-k selection (select.cu)
 enum PoolMode : int {

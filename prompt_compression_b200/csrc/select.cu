@@ -213,63 +213,79 @@ __device__ __forceinline__ int pow2_at_least(int x) {
 
 struct SelShared {
   float tile[kTile + 2 * kHaloMax];
-  union {
-    uint32_t hist[kBins];
-    unsigned long long cand[kListMax];   // (~key << 32) | index: ascending = key desc, index asc
-  } u;
+  uint32_t hist[kBins];
+  unsigned long long cand[kListMax];   // (~key << 32) | index: ascending = key desc, index asc
   int list[kListMax];
   int warp_tot[33];
   int s_bin, s_rem, n_a, n_b;
 };
 
-// General path (C > kListMax, or too many candidates in the threshold bin):
-// keys in the workspace, three radix levels, ordered ballot emission.
-__device__ __noinline__ void select_general(SelShared& sh, const float* __restrict__ s, int n, int r, int mode,
-                                            int C, uint32_t* __restrict__ keys, int* __restrict__ out) {
+// Calls f(j, valid, key_j) for every key of the row (keys padded to a
+// multiple of 4 per row, 16-byte aligned), warp-uniformly: each thread loads
+// four 16-byte vectors per round before using any of them.
+template <typename F>
+__device__ __forceinline__ void key_sweep(const uint32_t* __restrict__ keys, int n, F&& f) {
+  const uint4* kv = reinterpret_cast<const uint4*>(keys);
+  const int nv = (n + 3) / 4;
+  for (int base = 0; base < nv; base += 4 * kSelThreads) {
+    uint4 w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int vi = base + q * kSelThreads + threadIdx.x;
+      w[q] = vi < nv ? kv[vi] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = 4 * (base + q * kSelThreads + threadIdx.x);
+      f(j + 0, j + 0 < n, w[q].x);
+      f(j + 1, j + 1 < n, w[q].y);
+      f(j + 2, j + 2 < n, w[q].z);
+      f(j + 3, j + 3 < n, w[q].w);
+    }
+  }
+}
+
+// Warp-aggregated append of the lanes with pred to a shared list: returns
+// the lane's slot (or -1), one atomic per warp.
+__device__ __forceinline__ int warp_append(int* counter, bool pred) {
+  const uint32_t m = __ballot_sync(0xffffffffu, pred);
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  if (lane == 0 && m) base = atomicAdd(counter, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  return pred ? base + __popc(m & ((1u << lane) - 1u)) : -1;
+}
+
+// General path (C > kListMax, or more than kListMax keys share even a 24-bit
+// prefix with the C-th largest): three radix levels over the keys in the
+// workspace, then an ordered ballot emission.
+__device__ __noinline__ void select_general(SelShared& sh, int n, int C, const uint32_t* __restrict__ keys,
+                                            int* __restrict__ out) {
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
-  uint32_t* hist = sh.u.hist;
+  uint32_t* hist = sh.hist;
+  __syncthreads();
   for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0;
   __syncthreads();
-  pooled_sweep(s, n, r, mode, sh.tile, [&](int j, bool valid, float p) {
-    uint32_t bin = kBins;
-    if (valid) {
-      const uint32_t key = float_key(p);
-      keys[j] = key;
-      bin = key >> 20;
-    }
-    hist_add(hist, bin);
-  });
+  key_sweep(keys, n, [&](int, bool valid, uint32_t key) { hist_add(hist, valid ? key >> 20 : kBins); });
   __syncthreads();
   find_bin(hist, kBins, C, sh.warp_tot, &sh.s_bin, &sh.s_rem);
   uint32_t prefix = static_cast<uint32_t>(sh.s_bin);        // top 12 bits of T
   int remaining = sh.s_rem;
   for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0;
   __syncthreads();
-  for (int base = 0; base < n; base += kSelThreads) {
-    const int j = base + tid;
-    uint32_t bin = kBins;
-    if (j < n) {
-      const uint32_t key = keys[j];
-      if ((key >> 20) == prefix) bin = (key >> 8) & 4095u;
-    }
-    hist_add(hist, bin);
-  }
+  key_sweep(keys, n, [&](int, bool valid, uint32_t key) {
+    hist_add(hist, valid && (key >> 20) == prefix ? (key >> 8) & 4095u : kBins);
+  });
   __syncthreads();
   find_bin(hist, kBins, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
   prefix = (prefix << 12) | static_cast<uint32_t>(sh.s_bin);   // top 24 bits of T
   remaining = sh.s_rem;
   for (int b = tid; b < 256; b += kSelThreads) hist[b] = 0;
   __syncthreads();
-  for (int base = 0; base < n; base += kSelThreads) {
-    const int j = base + tid;
-    uint32_t bin = kBins;
-    if (j < n) {
-      const uint32_t key = keys[j];
-      if ((key >> 8) == prefix) bin = key & 255u;
-    }
-    hist_add(hist, bin);
-  }
+  key_sweep(keys, n, [&](int, bool valid, uint32_t key) {
+    hist_add(hist, valid && (key >> 8) == prefix ? key & 255u : kBins);
+  });
   __syncthreads();
   find_bin(hist, 256, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
   const uint32_t T = (prefix << 8) | static_cast<uint32_t>(sh.s_bin);
@@ -306,91 +322,17 @@ __device__ __noinline__ void select_general(SelShared& sh, const float* __restri
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads, 4)
-    topk_kernel(const float* __restrict__ scores, int n_cand, int pool_r, int pool_mode, int k, int n_tail,
-                int* __restrict__ idx, float* __restrict__ pooled, uint32_t* __restrict__ keys_ws) {
-  __shared__ SelShared sh;
-  const int u = blockIdx.x;
+// The candidates (sh.n_b <= kListMax of them) sorted by (key desc, index
+// asc) complete the selected list with `need` entries; the C indices are
+// then sorted ascending and written.
+__device__ __forceinline__ void finish_selection(SelShared& sh, int need, int C, int* __restrict__ out) {
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int n = n_cand;
-  const int C = k < n ? k : n;
-  const size_t out_len = static_cast<size_t>(C) + n_tail;
-  int* out = idx + static_cast<size_t>(u) * out_len;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-
-  // kept tail (the window)
-  for (int t = tid; t < n_tail; t += kSelThreads) out[C + t] = n + t;
-  if (C == 0 && pooled == nullptr) return;
-
-  const float* s = scores + static_cast<size_t>(u) * n;
-  uint32_t* keys = keys_ws + static_cast<size_t>(u) * n;
-  float* pout = pooled ? pooled + static_cast<size_t>(u) * n : nullptr;
-
-  // 1. pooled values -> (optional output) and the histogram of the keys' top 12 bits
-  for (int b = tid; b < kBins; b += kSelThreads) sh.u.hist[b] = 0;
-  if (tid == 0) { sh.n_a = 0; sh.n_b = 0; }
-  __syncthreads();
-  pooled_sweep(s, n, pool_r, pool_mode, sh.tile, [&](int j, bool valid, float p) {
-    uint32_t bin = kBins;
-    if (valid) {
-      if (pout) pout[j] = p;
-      bin = float_key(p) >> 20;
-    }
-    if (C > 0 && C < n) hist_add(sh.u.hist, bin);
-  });
-  if (C == 0) return;
-  if (C >= n) {
-    for (int j = tid; j < n; j += kSelThreads) out[j] = j;
-    return;
-  }
-  if (C > kListMax) {
-    __syncthreads();             // every thread is done with sweep 1's histogram
-    select_general(sh, s, n, pool_r, pool_mode, C, keys, out);
-    return;
-  }
-  __syncthreads();
-  find_bin(sh.u.hist, kBins, C, sh.warp_tot, &sh.s_bin, &sh.s_rem);
-  const uint32_t b1 = static_cast<uint32_t>(sh.s_bin);
-  const int need = sh.s_rem;     // keys of bin b1 still to take (>= 1)
-  __syncthreads();               // everyone has read the histogram: its memory now holds candidates
-
-  // 2. bins above b1 are selected; bin b1 holds the candidates
-  pooled_sweep(s, n, pool_r, pool_mode, sh.tile, [&](int j, bool valid, float p) {
-    const uint32_t key = valid ? float_key(p) : 0u;
-    const uint32_t bin = key >> 20;
-    const bool is_a = valid && bin > b1;
-    const bool is_b = valid && bin == b1;
-    const uint32_t ma = __ballot_sync(0xffffffffu, is_a);
-    const uint32_t mb = __ballot_sync(0xffffffffu, is_b);
-    int base_a = 0, base_b = 0;
-    if (lane == 0) {
-      if (ma) base_a = atomicAdd(&sh.n_a, __popc(ma));
-      if (mb) base_b = atomicAdd(&sh.n_b, __popc(mb));
-    }
-    base_a = __shfl_sync(0xffffffffu, base_a, 0);
-    base_b = __shfl_sync(0xffffffffu, base_b, 0);
-    if (is_a) sh.list[base_a + __popc(ma & lt_mask)] = j;   // fewer than C <= kListMax of these
-    if (is_b) {
-      const int pos = base_b + __popc(mb & lt_mask);
-      if (pos < kListMax)
-        sh.u.cand[pos] = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(j);
-    }
-  });
-  __syncthreads();
   const int n_a = sh.n_a, n_b = sh.n_b;
-  if (n_b > kListMax) {          // a long run of (nearly) equal values: the general path
-    __syncthreads();
-    select_general(sh, s, n, pool_r, pool_mode, C, keys, out);
-    return;
-  }
-
-  // 3. order the candidates, complete the selection, order the indices
   const int pb = pow2_at_least(n_b);
-  for (int t = n_b + tid; t < pb; t += kSelThreads) sh.u.cand[t] = ~0ull;
+  for (int t = n_b + tid; t < pb; t += kSelThreads) sh.cand[t] = ~0ull;
   __syncthreads();
-  bitonic_sort(sh.u.cand, pb);
-  for (int t = tid; t < need; t += kSelThreads) sh.list[n_a + t] = static_cast<int>(sh.u.cand[t] & 0xffffffffu);
+  bitonic_sort(sh.cand, pb);
+  for (int t = tid; t < need; t += kSelThreads) sh.list[n_a + t] = static_cast<int>(sh.cand[t] & 0xffffffffu);
   const int pc = pow2_at_least(C);
   for (int t = C + tid; t < pc; t += kSelThreads) sh.list[t] = 0x7fffffff;
   __syncthreads();
@@ -398,17 +340,117 @@ __global__ void __launch_bounds__(kSelThreads, 4)
   for (int t = tid; t < C; t += kSelThreads) out[t] = sh.list[t];
 }
 
+__global__ void __launch_bounds__(kSelThreads, 4)
+    topk_kernel(const float* __restrict__ scores, int n_cand, int pool_r, int pool_mode, int k, int n_tail,
+                int* __restrict__ idx, float* __restrict__ pooled, uint32_t* __restrict__ keys_ws, int key_stride) {
+  extern __shared__ __align__(16) uint8_t sel_smem[];   // 50 KB: above the 48 KB of static shared memory
+  SelShared& sh = *reinterpret_cast<SelShared*>(sel_smem);
+  const int u = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int n = n_cand;
+  const int C = k < n ? k : n;
+  const size_t out_len = static_cast<size_t>(C) + n_tail;
+  int* out = idx + static_cast<size_t>(u) * out_len;
+
+  // kept tail (the window)
+  for (int t = tid; t < n_tail; t += kSelThreads) out[C + t] = n + t;
+  if (C == 0 && pooled == nullptr) return;
+
+  const float* s = scores + static_cast<size_t>(u) * n;
+  uint32_t* keys = keys_ws + static_cast<size_t>(u) * key_stride;
+  float* pout = pooled ? pooled + static_cast<size_t>(u) * n : nullptr;
+  const bool select = C > 0 && C < n;
+
+  // 1. pooled values -> (optional output), keys to the workspace, histogram of their top 12 bits
+  for (int b = tid; b < kBins; b += kSelThreads) sh.hist[b] = 0;
+  if (tid == 0) { sh.n_a = 0; sh.n_b = 0; }
+  __syncthreads();
+  pooled_sweep(s, n, pool_r, pool_mode, sh.tile, [&](int j, bool valid, float p) {
+    uint32_t bin = kBins;
+    if (valid) {
+      if (pout) pout[j] = p;
+      const uint32_t key = float_key(p);
+      if (select) keys[j] = key;
+      bin = key >> 20;
+    }
+    if (select) hist_add(sh.hist, bin);
+  });
+  if (C == 0) return;
+  if (C >= n) {
+    for (int j = tid; j < n; j += kSelThreads) out[j] = j;
+    return;
+  }
+  __syncthreads();               // keys and histogram complete
+  if (C > kListMax) {
+    select_general(sh, n, C, keys, out);
+    return;
+  }
+  find_bin(sh.hist, kBins, C, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  const uint32_t b1 = static_cast<uint32_t>(sh.s_bin);
+  const int need1 = sh.s_rem;    // keys of bin b1 still to take (>= 1)
+  for (int b = tid; b < kBins; b += kSelThreads) sh.hist[b] = 0;
+  __syncthreads();
+
+  // 2. bins above b1 are selected; bin b1's keys are candidates, histogrammed on their next 12 bits
+  key_sweep(keys, n, [&](int j, bool valid, uint32_t key) {
+    const uint32_t bin = key >> 20;
+    const bool in_b = valid && bin == b1;
+    hist_add(sh.hist, in_b ? (key >> 8) & 4095u : kBins);
+    const int pa = warp_append(&sh.n_a, valid && bin > b1);   // fewer than C <= kListMax of these
+    if (pa >= 0) sh.list[pa] = j;
+    const int pb = warp_append(&sh.n_b, in_b);
+    if (pb >= 0 && pb < kListMax) sh.cand[pb] = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(j);
+  });
+  __syncthreads();
+  if (sh.n_b <= kListMax) {
+    finish_selection(sh, need1, C, out);
+    return;
+  }
+
+  // 3. too many candidates: refine bin b1 by the next 12 bits
+  find_bin(sh.hist, kBins, need1, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  const uint32_t p24 = (b1 << 12) | static_cast<uint32_t>(sh.s_bin);
+  const int need2 = sh.s_rem;
+  if (tid == 0) sh.n_b = 0;
+  __syncthreads();
+  key_sweep(keys, n, [&](int j, bool valid, uint32_t key) {
+    const uint32_t pre = key >> 8;
+    const int pa = warp_append(&sh.n_a, valid && (key >> 20) == b1 && pre > p24);
+    if (pa >= 0) sh.list[pa] = j;
+    const int pb = warp_append(&sh.n_b, valid && pre == p24);
+    if (pb >= 0 && pb < kListMax) sh.cand[pb] = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(j);
+  });
+  __syncthreads();
+  if (sh.n_b <= kListMax) {
+    finish_selection(sh, need2, C, out);
+    return;
+  }
+  select_general(sh, n, C, keys, out);   // long runs of equal values
+}
+
 }  // namespace
 
+// Keys of one row, padded to a multiple of four (16-byte vectors).
+static int key_stride(int n_cand) { return n_cand > 0 ? (n_cand + 3) & ~3 : 0; }
+
 size_t topk_ws_bytes(int units, int n_cand) {
-  return static_cast<size_t>(units) * static_cast<size_t>(n_cand > 0 ? n_cand : 0) * sizeof(uint32_t);
+  return static_cast<size_t>(units) * static_cast<size_t>(key_stride(n_cand)) * sizeof(uint32_t);
 }
 
 cudaError_t launch_topk(const float* scores, int units, int n_cand, int pool_mode, int pool_kernel, int k,
                         int n_tail, int* idx, float* pooled, void* ws, cudaStream_t stream) {
   if (units == 0) return cudaSuccess;
-  topk_kernel<<<units, kSelThreads, 0, stream>>>(scores, n_cand, pool_kernel / 2, pool_mode, k, n_tail, idx,
-                                                 pooled, static_cast<uint32_t*>(ws));
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(SelShared)));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  topk_kernel<<<units, kSelThreads, sizeof(SelShared), stream>>>(scores, n_cand, pool_kernel / 2, pool_mode, k, n_tail, idx,
+                                                 pooled, static_cast<uint32_t*>(ws), key_stride(n_cand));
   return cudaGetLastError();
 }
 
