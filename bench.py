@@ -456,8 +456,8 @@ def run_speckv(args, cfg, P, dev, world, rank, headline, prefill=False):
     flops_pass = algorithmic_flops(cfg)
     peak, _ = tensor_peak(peaks)
     kernels = {
-        "score_lse_pass": {"ms": per["score_lse_pass"],
-                           "tflops": flops_pass / (per["score_lse_pass"] * 1e-3) / 1e12},
+        launches[0][0]: {"ms": per[launches[0][0]],
+                         "tflops": flops_pass / (per[launches[0][0]] * 1e-3) / 1e12},
         "score_colsum_pass": {"ms": per["score_colsum_pass"],
                               "tflops": flops_pass / (per["score_colsum_pass"] * 1e-3) / 1e12},
         "topk_select": {"ms": per["topk_select"],
@@ -466,9 +466,7 @@ def run_speckv(args, cfg, P, dev, world, rank, headline, prefill=False):
                        "gbs": cfg.units * 4 * cfg.keep * cfg.head_dim * 2 / (per["kv_compact"] * 1e-3) / 1e9},
     }
     if prefill:
-        del kernels["score_lse_pass"]
-        kernels["prefill_attention"] = {"ms": per["prefill_attention"],
-                                        "tflops": prefill_flops(cfg) / (per["prefill_attention"] * 1e-3) / 1e12}
+        kernels["prefill_attention"]["tflops"] = prefill_flops(cfg) / (per["prefill_attention"] * 1e-3) / 1e12
     for name in ("score_lse_pass", "score_colsum_pass", "prefill_attention"):
         if name in kernels:
             kernels[name]["frac"] = kernels[name]["tflops"] / peak

@@ -48,11 +48,18 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Add one to hist[bin] for every lane with bin < kBins, one atomic per
-// distinct bin in the warp.
+// Add one to hist[bin] for every lane with bin < kBins.  Scores cluster, so
+// whole warps often share a bin: the lanes that match lane 0's bin add
+// together (one atomic), the others add their own.
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
-  const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-  if (bin < kBins && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+  const uint32_t b0 = __shfl_sync(0xffffffffu, bin, 0);
+  const uint32_t same = __ballot_sync(0xffffffffu, bin == b0);
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
+    if (b0 < kBins) atomicAdd(&hist[b0], __popc(same));
+  } else if (bin != b0 && bin < kBins) {
+    atomicAdd(&hist[bin], 1u);
+  }
 }
 
 // Exclusive prefix sum over the CTA (kSelThreads threads); also returns the total.
@@ -152,24 +159,29 @@ __device__ __forceinline__ void pooled_sweep(const float* __restrict__ s, int n,
   const int tid = threadIdx.x;
   const bool staged = r <= kHaloMax;
   const float pad = mode == POOL_MAX ? -INFINITY : 0.f;
+  const int len = kTile + 2 * r;
+  // scores[base - r, base + kTile + r) with padding outside [0, n); the next
+  // tile's loads are issued before this tile is pooled, so their latency
+  // overlaps the pooling
+  float v[kTileLoads];
+  auto load_tile = [&](int base) {
+#pragma unroll
+    for (int q = 0; q < kTileLoads; ++q) {
+      const int t = tid + q * kSelThreads;
+      const int jj = base - r + t;
+      v[q] = (t < len && jj >= 0 && jj < n) ? __ldg(s + jj) : pad;
+    }
+  };
+  if (staged) load_tile(0);
   for (int base = 0; base < n; base += kTile) {
     if (staged) {
-      // scores[base - r, base + kTile + r) with padding outside [0, n): all
-      // loads of a thread are issued before any of them is stored
-      const int len = kTile + 2 * r;
-      float v[kTileLoads];
-#pragma unroll
-      for (int q = 0; q < kTileLoads; ++q) {
-        const int t = tid + q * kSelThreads;
-        const int jj = base - r + t;
-        v[q] = (t < len && jj >= 0 && jj < n) ? __ldg(s + jj) : pad;
-      }
 #pragma unroll
       for (int q = 0; q < kTileLoads; ++q) {
         const int t = tid + q * kSelThreads;
         if (t < len) tile[t] = v[q];
       }
       __syncthreads();
+      if (base + kTile < n) load_tile(base + kTile);
     }
 #pragma unroll 1
     for (int i = 0; i < kTile / kSelThreads; ++i) {
@@ -395,7 +407,7 @@ __global__ void __launch_bounds__(kSelThreads, 4)
   key_sweep(keys, n, [&](int j, bool valid, uint32_t key) {
     const uint32_t bin = key >> 20;
     const bool in_b = valid && bin == b1;
-    hist_add(sh.hist, in_b ? (key >> 8) & 4095u : kBins);
+    if (in_b) atomicAdd(&sh.hist[(key >> 8) & 4095u], 1u);
     const int pa = warp_append(&sh.n_a, valid && bin > b1);   // fewer than C <= kListMax of these
     if (pa >= 0) sh.list[pa] = j;
     const int pb = warp_append(&sh.n_b, in_b);

@@ -345,8 +345,8 @@ def test_argument_errors_do_not_launch(P):
     assert e.value.status == P.binding.SPK_ERR_UNSUPPORTED
     q = torch.zeros((1, 1, 4, 8, 64), dtype=torch.bfloat16, device="cuda")
     k = torch.zeros((1, 1, 3, 64, 64), dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(P.SpeckvError) as e:
-        P.speckv_score(q, k, 4, s)
+    with pytest.raises(P.SpeckvError) as e:      # 3 KV heads: the shape is rejected by the library
+        P.speckv_score(q, k, 4, torch.zeros((3, 60), dtype=torch.float32, device="cuda"))
     assert e.value.status == P.binding.SPK_ERR_ARG
     k = torch.zeros((1, 1, 2, 64, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(P.SpeckvError) as e:
