@@ -55,9 +55,10 @@ def _load():
         lib.oracle_gather_rows.argtypes = [_u8p, I, I, _i32p, I, _u8p]
         lib.oracle_decode_row.argtypes = [_u16p, _u16p, _u16p, I, I, D, _dp]
         lib.oracle_prefill_row.argtypes = [_u16p, _u16p, _u16p, I, I, I, D, _dp, _dp]
+        lib.oracle_vs_row.argtypes = [_u16p, _u16p, _u16p, _u8p, _u8p, I, I, I, D, _dp, _dp]
         for f in (lib.oracle_speckv_unit, lib.oracle_speckv_unit_f64, lib.oracle_specpc_batch,
                   lib.oracle_specpc_batch_f64, lib.oracle_maxpool, lib.oracle_avgpool, lib.oracle_topk_with_tail,
-                  lib.oracle_gather_rows, lib.oracle_decode_row, lib.oracle_prefill_row):
+                  lib.oracle_gather_rows, lib.oracle_decode_row, lib.oracle_prefill_row, lib.oracle_vs_row):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -219,6 +220,36 @@ def prefill_unit(q, k, v, n_window: int, n_lookahead: int, n_in: int, scale: flo
                                           scale, _ptr(row, _dp), ctypes.byref(l)))
             out[h, i] = row
             lse[h * R + i] = l.value
+    return out, lse
+
+
+def vs_attention_unit(q, k, v, vertical, slash, scale: float = 1.0):
+    """Vertical-Slash sparse attention of one unit's query heads.
+
+    q [g, n_q, d]: the last n_q positions of the sequence (row i at
+    n - n_q + i); k, v [n, d]; vertical: key indices every row sees; slash:
+    offsets o = p - j every row sees (bf16 bit patterns for q, k, v).
+    Returns (out [g, n_q, d] float64, lse [g * n_q], natural log)."""
+    lib = _load()
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    g, n_q, d = q.shape
+    n = k.shape[0]
+    vm = np.zeros(n, np.uint8)
+    sm = np.zeros(n, np.uint8)
+    vm[np.asarray(vertical, np.int64)] = 1
+    sm[np.asarray(slash, np.int64)] = 1
+    out = np.zeros((g, n_q, d), np.float64)
+    lse = np.zeros(g * n_q, np.float64)
+    for h in range(g):
+        for i in range(n_q):
+            row = np.zeros(d, np.float64)
+            l = ctypes.c_double(0.0)
+            _check(lib.oracle_vs_row(_ptr(q[h, i], _u16p), _ptr(k, _u16p), _ptr(v, _u16p), _ptr(vm, _u8p),
+                                     _ptr(sm, _u8p), n, n - n_q + i, d, scale, _ptr(row, _dp), ctypes.byref(l)))
+            out[h, i] = row
+            lse[h * n_q + i] = l.value
     return out, lse
 
 

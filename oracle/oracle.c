@@ -356,3 +356,45 @@ int oracle_prefill_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     free(z);
     return 0;
 }
+
+/*
+ * Vertical-Slash sparse attention of one query row ("Draft-based Approximate
+ * Inference for LLMs", paper notes, section 损失函数 / 训练策略: SpecKV runs the
+ * target prefill with Vertical-Slash sparse attention; the pattern is the one
+ * of the cited sparse-attention work: a set V of key columns every row sees
+ * and a set S of diagonals, i.e. offsets o = p - j).  The row at position p
+ * attends to the keys j <= p with j in V, or p - j in S, or j = p (a token
+ * always sees itself, so every softmax is defined):
+ *   z_j = scale <q, k_j>,  out = sum_j softmax(z)_j v_j,  lse = log sum_j exp(z_j)
+ * over those keys.  vmask[j] / smask[o] (0 or 1, n entries each) mark V and S.
+ * q [d], k/v [n][d] as bf16 bit patterns; out [d], *lse in double.
+ */
+int oracle_vs_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint8_t *vmask,
+                  const uint8_t *smask, int n, int p, int d, double scale, double *out, double *lse) {
+    if (n < 1 || p < 0 || p >= n || d < 1) return -1;
+    double *z = (double *)malloc((size_t)(p + 1) * sizeof(double));
+    if (!z) return -1;
+    double zmax = -INFINITY;
+    for (int j = 0; j <= p; ++j) {
+        z[j] = -INFINITY;
+        if (!(j == p || vmask[j] || smask[p - j])) continue;
+        double dot = 0.0;
+        for (int t = 0; t < d; ++t) dot += bf16_to_double(q[t]) * bf16_to_double(k[(size_t)j * d + t]);
+        z[j] = scale * dot;
+        if (z[j] > zmax) zmax = z[j];
+    }
+    double den = 0.0;
+    for (int j = 0; j <= p; ++j) {
+        z[j] = (z[j] == -INFINITY) ? 0.0 : exp(z[j] - zmax);
+        den += z[j];
+    }
+    *lse = zmax + log(den);
+    for (int t = 0; t < d; ++t) out[t] = 0.0;
+    for (int j = 0; j <= p; ++j) {
+        if (z[j] == 0.0) continue;
+        const double pj = z[j] / den;
+        for (int t = 0; t < d; ++t) out[t] += pj * bf16_to_double(v[(size_t)j * d + t]);
+    }
+    free(z);
+    return 0;
+}
