@@ -167,6 +167,46 @@ spk_status speckv_prefill_attention(const spk_speckv_shape* shape, const void* q
                                    void* stream);
 
 /* ------------------------------------------------------------------------
+ * Vertical-Slash sparse prefill attention (section 损失函数 / 训练策略: SpecKV
+ * runs the target prefill with Vertical-Slash sparse attention, the pattern
+ * of the cited sparse-attention work)
+ *
+ * Per unit (batch element, layer, KV head) the pattern is a set of vertical
+ * key columns and a set of slash diagonals (offsets o = p - j).  The query
+ * row at position p attends to the keys j <= p with j in vertical, or
+ * p - j in slash, or j = p (a token always sees itself):
+ *   out[u*g + h][i] = softmax_j(scale * q . k_j) . v_j over those keys,
+ *   lse2[u*g + h][i] = log2 sum_j 2^(scale*log2(e) * q . k_j)   (optional)
+ * Query rows are the last n_q positions: row i sits at n - n_q + i.
+ *
+ *   q         bf16 [batch][layers][hq][n_q][head_dim]
+ *   k, v      bf16 [batch][layers][hkv][n][head_dim]
+ *   vertical  int32 [units][n_vertical], ascending, unique, in [0, n)
+ *   slash     int32 [units][n_slash], ascending, unique, in [0, n)
+ *   out       bf16 [batch][layers][hq][n_q][head_dim]
+ *   lse2      fp32 [units * g][n_q] or NULL
+ *   workspace vs_workspace_size(shape) bytes (the vertical keys' K and V rows,
+ *             gathered on the stream first), 16-byte aligned; may be NULL when
+ *             n_vertical = 0
+ * A vertical or slash entry outside [0, n) is ignored and recorded as
+ * SPK_ERR_ARG in the device error word; unsorted lists give wrong results.
+ * Probabilities enter the P.V product as bf16 (fp32 accumulation).
+ * Supported: head_dim in {64, 128}; hq % hkv == 0; 1 <= n_q <= n <= 131072;
+ * n_vertical <= 4096; n_slash <= n.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int batch, layers, hq, hkv, head_dim;
+  int n, n_q, n_vertical, n_slash;
+  float scale;
+} spk_vs_shape;
+
+size_t vs_workspace_size(const spk_vs_shape* shape);
+
+spk_status vs_sparse_attention(const spk_vs_shape* shape, const void* q_bf16, const void* k_bf16,
+                               const void* v_bf16, const int32_t* vertical, const int32_t* slash, void* out_bf16,
+                               float* lse2, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * SpecPC scoring (section 关键设计, SpecPC)
  *
  * Per batch element b, the draft's last W = n_rows query positions: row i sits

@@ -20,7 +20,7 @@ from .binding import (  # noqa: F401
     speckv_prefill_attention, specpc_workspace_size, specpc_score, specpc_row_offsets, specpc_colsum,
     topk_workspace_size, topk_select, kv_compact, decode_attention,
     spk_device_error, spk_selftest_wait_timeout, spk_exp2_fma, mapped_host_pointer,
-    SPK_POOL_MAX, SPK_POOL_AVG,
+    SPK_POOL_MAX, SPK_POOL_AVG, vs_workspace_size, vs_sparse_attention,
 )
 from .pipeline import speckv_compress, specpc_select, cascade_compress  # noqa: F401
 
@@ -30,5 +30,5 @@ __all__ = [
     "speckv_prefill_attention", "specpc_workspace_size", "specpc_score", "specpc_row_offsets", "specpc_colsum",
     "topk_workspace_size", "topk_select", "kv_compact", "decode_attention",
     "spk_device_error", "spk_selftest_wait_timeout", "spk_exp2_fma", "mapped_host_pointer",
-    "SPK_POOL_MAX", "SPK_POOL_AVG", "speckv_compress", "specpc_select", "cascade_compress",
+    "SPK_POOL_MAX", "SPK_POOL_AVG", "vs_workspace_size", "vs_sparse_attention", "speckv_compress", "specpc_select", "cascade_compress",
 ]

@@ -44,6 +44,12 @@ class SpecpcShape(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
+class VsShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("layers", ctypes.c_int), ("hq", ctypes.c_int),
+                ("hkv", ctypes.c_int), ("head_dim", ctypes.c_int), ("n", ctypes.c_int), ("n_q", ctypes.c_int),
+                ("n_vertical", ctypes.c_int), ("n_slash", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -59,6 +65,7 @@ def load_library():
     vp, sz, I, F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
     sk = ctypes.POINTER(SpeckvShape)
     sp = ctypes.POINTER(SpecpcShape)
+    vsp = ctypes.POINTER(VsShape)
     sig = {
         "speckv_workspace_size": (sz, [sk]),
         "speckv_score": (I, [sk, vp, vp, vp, vp, vp, sz, vp]),
@@ -80,6 +87,8 @@ def load_library():
         "spk_exp2_fma": (I, [vp, vp, I, vp]),
         "spk_mapped_host_pointer": (I, [vp, ctypes.POINTER(vp)]),
         "decode_attention": (I, [I, I, I, I, I, I, F, vp, vp, vp, vp, vp]),
+        "vs_workspace_size": (sz, [vsp]),
+        "vs_sparse_attention": (I, [vsp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -397,6 +406,52 @@ def decode_attention(q, k, v, out=None, scale: float = 1.0, stream=None):
     _check(lib.decode_attention(Bsz, L, hq, hkv, d, n_kv, float(scale), _dev(q, "q", torch.bfloat16),
                                 _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
                                 _dev(out, "out", torch.float32), _stream(stream)))
+    return out
+
+
+# --------------------------------------------------------------------- Vertical-Slash sparse prefill
+def vs_shape(q, k, n_vertical: int, n_slash: int, scale: float = 1.0) -> VsShape:
+    if q.dim() != 5 or k.dim() != 5:
+        raise ValueError("q is [B, L, Hq, n_q, d] and k is [B, L, Hkv, n, d]")
+    B, L, hq, n_q, d = q.shape
+    Bk, Lk, hkv, n, dk = k.shape
+    if (B, L, d) != (Bk, Lk, dk):
+        raise ValueError("q and k disagree on batch, layers or head_dim")
+    return VsShape(B, L, hq, hkv, d, n, n_q, n_vertical, n_slash, float(scale))
+
+
+def vs_workspace_size(shape: VsShape) -> int:
+    return int(load_library().vs_workspace_size(ctypes.byref(shape)))
+
+
+def vs_sparse_attention(q, k, v, vertical, slash, out=None, lse2=None, workspace=None, scale: float = 1.0,
+                        stream=None):
+    """Vertical-Slash sparse attention: q [B, L, Hq, n_q, d] (the last n_q
+    positions), k, v [B, L, Hkv, n, d]; vertical int32 [units, n_v] and slash
+    int32 [units, n_s] (ascending) per unit = (b, layer, KV head).  Returns
+    out bf16 [B, L, Hq, n_q, d]; fills lse2 (fp32 [B*L*Hq, n_q]) when given."""
+    lib = load_library()
+    if vertical is None or slash is None or vertical.dim() < 1 or slash.dim() < 1:
+        raise ValueError("vertical and slash are int32 [units, count] tensors")
+    n_v, n_s = vertical.shape[-1], slash.shape[-1]
+    shape = vs_shape(q, k, n_v, n_s, scale)
+    units = shape.batch * shape.layers * shape.hkv
+    if tuple(v.shape) != tuple(k.shape):
+        raise ValueError("v must have k's shape")
+    _numel(vertical, "vertical", units * n_v)
+    _numel(slash, "slash", units * n_s)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    _numel(out, "out", q.numel())
+    _numel(lse2, "lse2", shape.batch * shape.layers * shape.hq * shape.n_q, required=False)
+    ws = None
+    if n_v > 0:
+        ws = _workspace(workspace, vs_workspace_size(shape), q.device, stream)
+    _check(lib.vs_sparse_attention(ctypes.byref(shape), _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
+                                   _dev(v, "v", torch.bfloat16), _dev(vertical, "vertical", torch.int32),
+                                   _dev(slash, "slash", torch.int32), _dev(out, "out", torch.bfloat16),
+                                   _dev(lse2, "lse2", torch.float32), _dev(ws, "workspace"),
+                                   ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
     return out
 
 

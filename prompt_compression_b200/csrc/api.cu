@@ -309,6 +309,89 @@ spk_status speckv_prefill_attention(const spk_speckv_shape* s, const void* q, co
   return ok();
 }
 
+// ------------------------------------------------------------------ Vertical-Slash sparse prefill
+static spk_status check_vs(const spk_vs_shape* s, long long& units) {
+  if (s == nullptr) return fail(SPK_ERR_ARG, "shape is NULL");
+  if (s->batch < 1 || s->layers < 1 || s->hq < 1 || s->hkv < 1 || s->n < 1 || s->n_q < 1)
+    return fail(SPK_ERR_ARG, "batch, layers, hq, hkv, n and n_q must be >= 1");
+  if (s->hq % s->hkv != 0) return fail(SPK_ERR_ARG, "hq (%d) must be a multiple of hkv (%d)", s->hq, s->hkv);
+  if (s->n_q > s->n) return fail(SPK_ERR_ARG, "n_q must be <= n");
+  if (s->n_vertical < 0 || s->n_slash < 0) return fail(SPK_ERR_ARG, "n_vertical and n_slash must be >= 0");
+  if (!(s->scale > 0.f) || !std::isfinite(s->scale)) return fail(SPK_ERR_ARG, "scale must be finite and > 0");
+  if (s->head_dim != 64 && s->head_dim != 128)
+    return fail(SPK_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", s->head_dim);
+  if (s->n > kVsMaxN) return fail(SPK_ERR_UNSUPPORTED, "n = %d exceeds %d", s->n, kVsMaxN);
+  if (s->n_vertical > kVsMaxVert) return fail(SPK_ERR_UNSUPPORTED, "n_vertical = %d exceeds %d", s->n_vertical, kVsMaxVert);
+  if (s->n_slash > s->n) return fail(SPK_ERR_ARG, "n_slash must be <= n");
+  units = static_cast<long long>(s->batch) * s->layers * s->hkv;
+  const long long items = units * (s->hq / s->hkv) * ((s->n_q + 127) / 128);
+  if (items > 0x7fffffffLL || units * (s->hq / s->hkv) > 0x7fffffffLL) return fail(SPK_ERR_UNSUPPORTED, "too many units");
+  return SPK_OK;
+}
+
+size_t vs_workspace_size(const spk_vs_shape* s) {
+  long long units;
+  if (check_vs(s, units) != SPK_OK) return 0;
+  return round_up(2 * static_cast<size_t>(units) * s->n_vertical * s->head_dim * 2, 256);
+}
+
+spk_status vs_sparse_attention(const spk_vs_shape* s, const void* q, const void* k, const void* v,
+                               const int32_t* vertical, const int32_t* slash, void* out, float* lse2, void* ws,
+                               size_t ws_bytes, void* stream) {
+  long long units;
+  spk_status st = check_vs(s, units);
+  if (st != SPK_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr)
+    return fail(SPK_ERR_ARG, "q, k, v and out must be non-NULL device pointers");
+  if ((s->n_vertical > 0 && vertical == nullptr) || (s->n_slash > 0 && slash == nullptr))
+    return fail(SPK_ERR_ARG, "vertical / slash must be non-NULL when their counts are > 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SPK_ERR_ARG, "q, k, v and out must be 16-byte aligned");
+  const size_t need = vs_workspace_size(s);
+  if (s->n_vertical > 0) {
+    if (ws == nullptr || ws_bytes < need)
+      return fail(SPK_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : 0);
+    if (!aligned16(ws)) return fail(SPK_ERR_ARG, "workspace must be 16-byte aligned");
+  }
+  const int g = s->hq / s->hkv;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* kvert = static_cast<uint8_t*>(ws);
+  uint8_t* vvert = kvert + static_cast<size_t>(units) * s->n_vertical * s->head_dim * 2;
+  CUtensorMap maps[5];
+  if ((st = make_map(&maps[0], q, s->head_dim, s->n_q, units * g)) != SPK_OK) return st;
+  if ((st = make_map(&maps[1], k, s->head_dim, s->n, units)) != SPK_OK) return st;
+  if ((st = make_map(&maps[2], v, s->head_dim, s->n, units)) != SPK_OK) return st;
+  if (s->n_vertical > 0) {
+    if ((st = make_map(&maps[3], kvert, s->head_dim, s->n_vertical, units)) != SPK_OK) return st;
+    if ((st = make_map(&maps[4], vvert, s->head_dim, s->n_vertical, units)) != SPK_OK) return st;
+    // the vertical keys' K and V rows, gathered once per unit (indices checked on the device)
+    cudaError_t e = launch_compact(k, v, static_cast<int>(units), s->n, s->head_dim * 2, vertical, s->n_vertical, 1,
+                                   kvert, vvert, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "vertical gather launch");
+  } else {
+    maps[3] = maps[1];   // never read: no vertical tiles
+    maps[4] = maps[2];
+  }
+  VsParams p;
+  memset(&p, 0, sizeof p);
+  p.n = s->n;
+  p.n_q = s->n_q;
+  p.g = g;
+  p.n_v = s->n_vertical;
+  p.n_s = s->n_slash;
+  p.c2 = s->scale * 1.4426950408889634f;
+  p.row_blocks = (s->n_q + 127) / 128;
+  p.n_items = static_cast<int>(units * g * p.row_blocks);
+  p.vert = vertical;
+  p.slash = slash;
+  p.out = out;
+  p.lse2 = lse2;
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  cudaError_t e = launch_vs_attn(s->head_dim, maps, p, grid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "Vertical-Slash attention launch");
+  return ok();
+}
+
 // ------------------------------------------------------------------ SpecPC
 static spk_status check_specpc(const spk_specpc_shape* s, SpeckvGeom& g) {
   if (s == nullptr) return fail(SPK_ERR_ARG, "shape is NULL");

@@ -94,6 +94,26 @@ struct AttnParams {
 cudaError_t launch_attn(int head_dim, const CUtensorMap (&maps)[5], const AttnParams& p, int grid,
                         cudaStream_t stream);
 
+// Vertical-Slash sparse prefill attention (vs.cu)
+constexpr int kVsMaxN = 131072;     // keys per unit (the pattern's bitmaps live in shared memory)
+constexpr int kVsMaxVert = 4096;    // vertical columns per unit
+struct VsParams {
+  int n;             // keys per unit
+  int n_q;           // query rows per head: positions n - n_q .. n - 1
+  int g;             // query heads per unit
+  int n_v, n_s;      // vertical columns and slash offsets per unit
+  float c2;          // scale * log2(e)
+  int row_blocks;    // ceil(n_q / 128)
+  int n_items;       // units * g * row_blocks
+  const int* vert;   // [units][n_v] ascending key indices
+  const int* slash;  // [units][n_s] ascending offsets
+  void* out;         // bf16 [units * g][n_q][d]
+  float* lse2;       // fp32 [units * g][n_q] or null
+};
+// maps: q [units*g][n_q][d], k and v [units][n][d], gathered vertical k and v [units][n_v][d]
+cudaError_t launch_vs_attn(int head_dim, const CUtensorMap (&maps)[5], const VsParams& p, int grid,
+                           cudaStream_t stream);
+
 // pooling + top-k selection (select.cu)
 enum PoolMode : int {
   POOL_MAX = 0,   // max over the clipped window

@@ -1,0 +1,564 @@
+// vs.cu -- Vertical-Slash sparse prefill attention on tcgen05.
+//
+// "Draft-based Approximate Inference for LLMs" (paper notes), section
+// 损失函数 / 训练策略: SpecKV runs the target model's prefill with
+// Vertical-Slash sparse attention (the pattern of the cited sparse-attention
+// work).  Per unit (batch element, layer, KV head) the pattern is a sorted
+// set V of key columns and a sorted set S of diagonals (offsets o = p - j);
+// the query row at position p attends to the keys j <= p with j in V, or
+// p - j in S, or j = p (the token itself):
+//   out = softmax_j(scale q.k_j) . v_j over those keys (bf16), lse2 (optional,
+//   log2 domain) of the same sum.
+// Query rows are the last n_q positions of the n-token sequence, every query
+// head of the unit's GQA group.
+//
+// Work decomposition: an item is one query head's 128-row tile (positions
+// p0 .. p0 + 127).  Its keys come in 128-key tiles of two kinds:
+//   slash tiles    -- tiles of K/V that a slash diagonal (or the self
+//                     diagonal) crosses for some row of the item: tile t is
+//                     crossed iff some o in S u {0} lies in
+//                     [p0 - 128 t - 127, p_last - 128 t]; found by one walk
+//                     over S from the diagonal tile down;
+//   vertical tiles -- the vertical keys <= p_last, gathered beforehand into a
+//                     contiguous [units][n_v][d] buffer (kv_compact).
+// Masks are exact: in a slash tile key j is visible iff j <= p and (j = p or
+// j in V or p - j in S), from bitmaps of V and S in shared memory (one 32-bit
+// word per 32 keys, the slash word bit-reversed); in a vertical tile a key is
+// visible iff j <= p and its K/V tile was not a slash tile of the item (there
+// it was already counted).  The pipeline is the prefill attention's: a TMA
+// producer warp, a single-thread UMMA issuer (S = Q K^T from shared memory,
+// O += P V with P in TMEM as bf16 and V MN-major from shared memory) and
+// four softmax warps (thread = row; lazy rescale of O when the running max
+// moves by more than 2^8).  Every role derives the same tile sequence.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "score.cuh"
+
+namespace spk {
+namespace {
+
+constexpr int kVsSoftmaxWarps = 4;
+constexpr int kVsProducerWarp = 4;
+constexpr int kVsMmaWarp = 5;
+constexpr int kVsThreads = 6 * 32;
+constexpr float kVsRescale = 8.f;
+
+template <int D>
+struct VsCfg {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kAtoms = D / 64;
+  static constexpr int kStages = 2;
+  static constexpr int kBitWords = kVsMaxN / 32;
+  static constexpr int kSmemBytes = 1024 + kTileBytes + 2 * kStages * kTileBytes + 2 * kBitWords * 4 + kVsMaxVert * 4;
+  static_assert(kSmemBytes <= 227 * 1024 - 2048, "fits one CTA");
+};
+
+__device__ __forceinline__ uint64_t vs_mnmajor_desc(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void vs_tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t vs_pack_bf16(float lo, float hi) {
+  const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return a | (b << 16);
+}
+
+__device__ __forceinline__ int vs_site(int role, int which) { return 400 + role * 10 + which; }
+
+
+// The next slash tile of an item, walking down from tile t: tile t is crossed
+// iff some offset o in S u {0} lies in [p0 - 128 t - 127, p_last - 128 t].
+// a indexes the first offset of S (ascending) not below the window's lower
+// end, which only grows as t falls.  Returns -1 when no tile is left.
+__device__ __forceinline__ int next_slash_tile(const int* __restrict__ S, int n_s, int p0, int p_last, int& t,
+                                               int& a) {
+  while (t >= 0) {
+    const int lo = p0 - 128 * t - 127, hi = p_last - 128 * t;
+    while (a < n_s && __ldg(S + a) < lo) ++a;
+    const bool hit = (lo <= 0 && 0 <= hi) || (a < n_s && __ldg(S + a) <= hi);
+    const int cur = t--;
+    if (hit) return cur;
+  }
+  return -1;
+}
+
+// Number of entries of the ascending array x[0, n) that are <= v.
+__device__ __forceinline__ int upper_bound_le(const int* x, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (x[mid] <= v) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int upper_bound_le_global(const int* __restrict__ x, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(x + mid) <= v) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// 32 bits of a bitmap starting at bit o (bits below 0 and at or above
+// n_bits read as 0).
+__device__ __forceinline__ uint32_t bits32(const uint32_t* bm, int n_words, int o) {
+  if (o <= -32) return 0u;
+  if (o < 0) return n_words > 0 ? bm[0] << (-o) : 0u;
+  const int w = o >> 5, sh = o & 31;
+  const uint32_t lo = w < n_words ? bm[w] : 0u;
+  if (sh == 0) return lo;
+  const uint32_t hi = w + 1 < n_words ? bm[w + 1] : 0u;
+  return (lo >> sh) | (hi << (32 - sh));
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kVsThreads, 1)
+    vs_attn_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kvmap,
+                   const __grid_constant__ CUtensorMap vvmap, const VsParams p) {
+  using C = VsCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* const Q_s = smem;
+  uint8_t* const K_s = smem + C::kTileBytes;
+  uint8_t* const V_s = K_s + C::kStages * C::kTileBytes;
+  uint32_t* const vbits = reinterpret_cast<uint32_t*>(V_s + C::kStages * C::kTileBytes);   // V as a bitmap
+  uint32_t* const sbits = vbits + C::kBitWords;                                           // S as a bitmap
+  int* const vidx_s = reinterpret_cast<int*>(sbits + C::kBitWords);                      // V, ascending
+
+  __shared__ __align__(8) uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
+      p_full[2], pv_done, o_empty, done_bar, soft_bar;
+  __shared__ uint32_t slash_tiles[kVsMaxN / 128 / 32];   // tiles of the current item that were slash tiles
+  __shared__ uint32_t tmem_holder;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n = p.n;
+  const int n_words = (n + 31) >> 5;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kVsSoftmaxWarps);
+    }
+    mbar_init(&pv_done, 1);
+    mbar_init(&o_empty, kVsSoftmaxWarps);
+    mbar_init(&done_bar, 1);
+    mbar_init(&soft_bar, kVsSoftmaxWarps);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kVsMmaWarp) {
+    tmem_alloc(&tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == kVsProducerWarp && lane == 0) {
+    tma_prefetch_map(&qmap);
+    tma_prefetch_map(&kmap);
+    tma_prefetch_map(&vmap);
+    if (p.n_v > 0) {
+      tma_prefetch_map(&kvmap);
+      tma_prefetch_map(&vvmap);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_holder;
+  volatile int* abort_v = &abort_flag;
+
+  // item -> (unit, query head of the group, row block); rows' positions p0 .. p_last
+  auto item_geom = [&](int item, int& u, int& qh, int& rb, int& p0, int& p_last) {
+    rb = item % p.row_blocks;
+    const int hu = item / p.row_blocks;   // u * g + head
+    u = hu / p.g;
+    qh = hu;
+    p0 = n - p.n_q + rb * 128;
+    p_last = n - p.n_q + min(rb * 128 + 127, p.n_q - 1);
+  };
+  // tiles of an item: its slash tiles, then ceil(cv / 128) vertical tiles
+  auto count_tiles = [&](int u, int p0, int p_last, int& n_slash, int& cv) {
+    const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
+    int t = p_last >> 7, a = 0;
+    n_slash = 0;
+    while (next_slash_tile(S, p.n_s, p0, p_last, t, a) >= 0) ++n_slash;
+    cv = p.n_v > 0 ? upper_bound_le_global(p.vert + static_cast<size_t>(u) * p.n_v, p.n_v, p_last) : 0;
+    return n_slash + (cv + 127) / 128;
+  };
+
+  if (warp == kVsProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t tile_count = 0;
+      int items_done = 0;
+      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1}, q_last = -1;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
+        int u, qh, rb, p0, p_last;
+        item_geom(item, u, qh, rb, p0, p_last);
+        int n_slash, cv;
+        const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
+        if (!(ok = mbar_wait(&q_empty, (items_done & 1) ^ 1, abort_v, vs_site(0, 0)))) break;
+        mbar_arrive_expect_tx(&q_full, C::kTileBytes);
+        for (int a = 0; a < C::kAtoms; ++a) tma_load_3d(Q_s + a * 16384, &qmap, &q_full, a * 64, rb * 128, qh);
+        q_last = items_done & 1;
+        const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
+        int t = p_last >> 7, sa = 0;
+        for (int i = 0; ok && i < n_tiles; ++i, ++tile_count) {
+          const int st = tile_count & 1;
+          const uint32_t ph = (tile_count >> 1) & 1;
+          const bool slash = i < n_slash;
+          const int row0 = slash ? 128 * next_slash_tile(S, p.n_s, p0, p_last, t, sa) : 128 * (i - n_slash);
+          if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, abort_v, vs_site(0, 1)))) break;
+          mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+          for (int a = 0; a < C::kAtoms; ++a)
+            tma_load_3d(K_s + st * C::kTileBytes + a * 16384, slash ? &kmap : &kvmap, &k_full[st], a * 64, row0, u);
+          k_last[st] = static_cast<int>(ph);
+          if (!(ok = mbar_wait(&v_empty[st], ph ^ 1, abort_v, vs_site(0, 2)))) break;
+          mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
+          for (int a = 0; a < C::kAtoms; ++a)
+            tma_load_3d(V_s + st * C::kTileBytes + a * 16384, slash ? &vmap : &vvmap, &v_full[st], a * 64, row0, u);
+          v_last[st] = static_cast<int>(ph);
+        }
+      }
+      if (!ok) {
+        volatile int never = 0;
+        if (q_last >= 0) mbar_wait(&q_full, q_last, &never, vs_site(0, 7), 100000000ull);
+        for (int s = 0; s < 2; ++s) {
+          if (k_last[s] >= 0) mbar_wait(&k_full[s], k_last[s], &never, vs_site(0, 8), 100000000ull);
+          if (v_last[s] >= 0) mbar_wait(&v_full[s], v_last[s], &never, vs_site(0, 9), 100000000ull);
+        }
+      }
+    }
+  } else if (warp == kVsMmaWarp) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t T = 0;
+      int items_done = 0;
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 64) | (1u << 16);   // B (V) MN-major
+      const uint64_t q_desc = sw128_kmajor_desc(smem_u32(Q_s));
+      auto issue_s = [&](uint32_t Ti) -> bool {
+        const int st = Ti & 1;
+        if (!mbar_wait(&k_full[st], (Ti >> 1) & 1, abort_v, vs_site(1, 1))) return false;
+        tc_fence_after();
+        const uint64_t k_desc = sw128_kmajor_desc(smem_u32(K_s + st * C::kTileBytes));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_bf16_ss(tmem_base + st * 128, q_desc + koff, k_desc + koff, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[st]);
+        umma_commit(&k_empty[st]);
+        return true;
+      };
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
+        int u, qh, rb, p0, p_last;
+        item_geom(item, u, qh, rb, p0, p_last);
+        int n_slash, cv;
+        const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
+        if (!(ok = mbar_wait(&q_full, items_done & 1, abort_v, vs_site(1, 0)))) break;
+        if (T >= 1 && !(ok = mbar_wait(&pv_done, (T - 1) & 1, abort_v, vs_site(1, 2)))) break;
+        if (!(ok = issue_s(T))) break;
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          const uint32_t Tc = T + t;
+          if (t + 1 < n_tiles) {
+            if (Tc >= 1 && !(ok = mbar_wait(&pv_done, (Tc - 1) & 1, abort_v, vs_site(1, 3)))) break;
+            if (!(ok = issue_s(Tc + 1))) break;
+          }
+          const int st = Tc & 1;
+          if (!(ok = mbar_wait(&p_full[st], (Tc >> 1) & 1, abort_v, vs_site(1, 4)))) break;
+          if (!(ok = mbar_wait(&v_full[st], (Tc >> 1) & 1, abort_v, vs_site(1, 5)))) break;
+          if (t == 0 && items_done > 0 && !(ok = mbar_wait(&o_empty, (items_done - 1) & 1, abort_v, vs_site(1, 6))))
+            break;
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(V_s + st * C::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int a = 0; a < C::kAtoms; ++a) {
+              const uint64_t v_desc = vs_mnmajor_desc(v_base + a * 16384 + kk * 2048, 16384);
+              umma_bf16_ts(tmem_base + 256 + a * 64, tmem_base + st * 128 + kk * 8, v_desc, idesc_pv,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&v_empty[st]);
+          umma_commit(&pv_done);
+        }
+        if (!ok) break;
+        umma_commit(&q_empty);
+        T += n_tiles;
+      }
+      umma_commit(&done_bar);
+      volatile int never = 0;
+      mbar_wait(&done_bar, 0, &never, vs_site(1, 9), 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int tid = threadIdx.x;                        // 0 .. 127
+    const int r = warp * 32 + lane;                     // row within the Q tile = TMEM lane
+    const uint32_t tlane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    bool ok = true;
+    uint32_t T = 0;
+    int items_done = 0, loaded_unit = -1;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, int which) -> bool {
+      bool w = mbar_wait(bar, parity, abort_v, vs_site(2, which));
+      return __all_sync(0xffffffffu, w);
+    };
+    // the four softmax warps meet (their shared-memory writes before it are
+    // visible after it); a bounded wait, so an aborted CTA cannot strand a warp
+    uint32_t soft_phase = 0;
+    auto softmax_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&soft_bar);
+      const bool w = wait_all(&soft_bar, soft_phase, 4);
+      soft_phase ^= 1u;
+      return w;
+    };
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
+      int u, qh, rb, p0, p_last;
+      item_geom(item, u, qh, rb, p0, p_last);
+      int n_slash, cv;
+      const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
+      // this unit's pattern as bitmaps (and V as a list), and no slash tile yet
+      if (!(ok = softmax_sync())) break;                // the previous item is done with them
+      if (u != loaded_unit) {
+        for (int w = tid; w < n_words; w += 128) { vbits[w] = 0u; sbits[w] = 0u; }
+        if (!(ok = softmax_sync())) break;
+        const int* vg = p.vert + static_cast<size_t>(u) * p.n_v;
+        const int* sg = p.slash + static_cast<size_t>(u) * p.n_s;
+        for (int x = tid; x < p.n_v; x += 128) {
+          const int j = __ldg(vg + x);
+          vidx_s[x] = j;
+          if (j >= 0 && j < n) atomicOr(&vbits[j >> 5], 1u << (j & 31));
+          else record_error(SPK_DEVERR_INDEX, u);
+        }
+        for (int x = tid; x < p.n_s; x += 128) {
+          const int o = __ldg(sg + x);
+          if (o >= 0 && o < n) atomicOr(&sbits[o >> 5], 1u << (o & 31));
+          else record_error(SPK_DEVERR_INDEX, u);
+        }
+        loaded_unit = u;
+      }
+      for (int w = tid; w < kVsMaxN / 128 / 32; w += 128) slash_tiles[w] = 0u;
+      if (!(ok = softmax_sync())) break;
+
+      const int i_row = rb * 128 + r;
+      const bool live = i_row < p.n_q;
+      const int pos = live ? n - p.n_q + i_row : n - 1;
+      const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
+      int wt = p_last >> 7, wa = 0;                     // this role's walk over the slash tiles
+      float m = -INFINITY, l = 0.f;
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        const uint32_t Tc = T + t;
+        const int buf = Tc & 1;
+        const bool slash = t < n_slash;
+        int j0 = 0;
+        if (slash) {
+          const int tile = next_slash_tile(S, p.n_s, p0, p_last, wt, wa);
+          j0 = tile * 128;
+          if (lane == 0) atomicOr(&slash_tiles[tile >> 5], 1u << (tile & 31));   // read back by this warp only
+        }
+        // visibility of the tile's 128 keys for this row, 32 per word
+        uint32_t vis[4];
+        if (slash) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int jc = j0 + 32 * c;
+            const int rel = pos - jc;                   // key jc + b is causal iff b <= rel
+            const uint32_t causal = rel < 0 ? 0u : (rel >= 31 ? 0xffffffffu : ((2u << rel) - 1u));
+            const uint32_t self = (rel >= 0 && rel < 32) ? (1u << rel) : 0u;
+            const uint32_t vw = (jc >> 5) < n_words ? vbits[jc >> 5] : 0u;
+            const uint32_t sw = __brev(bits32(sbits, n_words, pos - jc - 31));
+            vis[c] = (vw | sw | self) & causal;
+          }
+        } else {
+          const int base = 128 * (t - n_slash);         // gathered rows of this vertical tile
+          const int cnt = min(128, cv - base);
+          __syncwarp();
+          // keys of slash tiles were counted there; vertical keys <= pos only
+          const int vis_n = upper_bound_le(vidx_s + base, cnt, pos);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int x = 32 * c + lane;
+            bool okc = false;
+            if (x < cnt) {
+              const int j = vidx_s[base + x];
+              okc = j >= 0 && j < n && !((slash_tiles[j >> 12] >> ((j >> 7) & 31)) & 1u);
+            }
+            const uint32_t dedupe = __ballot_sync(0xffffffffu, okc);
+            const int lim = vis_n - 32 * c;
+            const uint32_t pre = lim <= 0 ? 0u : (lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u));
+            vis[c] = dedupe & pre;
+          }
+        }
+        if (!(ok = wait_all(&s_full[buf], (Tc >> 1) & 1, 0))) break;
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t a0[32], a1[32];
+          tmem_ld32(tlane + buf * 128, a0);
+          tmem_ld32(tlane + buf * 128 + 32, a1);
+          tmem_ld_wait2(a0, a1);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            s[k] = ((vis[0] >> k) & 1u) ? __uint_as_float(a0[k]) : -INFINITY;
+            s[32 + k] = ((vis[1] >> k) & 1u) ? __uint_as_float(a1[k]) : -INFINITY;
+          }
+          tmem_ld32(tlane + buf * 128 + 64, a0);
+          tmem_ld32(tlane + buf * 128 + 96, a1);
+          tmem_ld_wait2(a0, a1);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            s[64 + k] = ((vis[2] >> k) & 1u) ? __uint_as_float(a0[k]) : -INFINITY;
+            s[96 + k] = ((vis[3] >> k) & 1u) ? __uint_as_float(a1[k]) : -INFINITY;
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 128; k += 4) mx = fmaxf(mx, max3f(s[k], s[k + 1], fmaxf(s[k + 2], s[k + 3])));
+        const float mt = mx * p.c2;
+        const bool need = mx != -INFINITY && mt > m + kVsRescale;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m - mt) : 1.f;
+          if (t > 0) {
+            if (!(ok = wait_all(&pv_done, (Tc - 1) & 1, 1))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t o[32];
+              tmem_ld32(tlane + 256 + ch * 32, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              vs_tmem_st32(tlane + 256 + ch * 32, o);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          }
+          if (need) {
+            l *= alpha;
+            m = mt;
+          }
+        }
+        // P = 2^(c2 s - m): masked keys (s = -inf) give 0; a row that has
+        // seen no key yet (m = -inf) has only masked keys here
+        const float mm = m == -INFINITY ? 0.f : m;
+        float sum0 = 0.f, sum1 = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          const float e0 = ex2_approx(fmaf(s[2 * k], p.c2, -mm));
+          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.c2, -mm));
+          sum0 += e0;
+          sum1 += e1;
+          pk[k] = vs_pack_bf16(e0, e1);
+        }
+        l += sum0 + sum1;
+        {
+          uint32_t (&p0r)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+          uint32_t (&p1r)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+          vs_tmem_st32(tlane + buf * 128, p0r);
+          vs_tmem_st32(tlane + buf * 128 + 32, p1r);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[buf]);
+      }
+      if (!ok) break;
+      const uint32_t Tl = T + n_tiles - 1;
+      if (Tl >= 1 && !(ok = wait_all(&pv_done, (Tl - 1) & 1, 2))) break;
+      if (!(ok = wait_all(&pv_done, Tl & 1, 3))) break;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                            (static_cast<size_t>(qh) * p.n_q + (live ? i_row : 0)) * D;
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tlane + 256 + ch * 32, o);
+        tmem_ld_wait(o);
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = vs_pack_bf16(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+            w.y = vs_pack_bf16(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+            w.z = vs_pack_bf16(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+            w.w = vs_pack_bf16(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+            dst[v4] = w;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty);
+      if (p.lse2 != nullptr && live) p.lse2[static_cast<size_t>(qh) * p.n_q + i_row] = m + lg2_approx(l);
+      T += n_tiles;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kVsMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int D>
+static cudaError_t vs_launch_one(const CUtensorMap (&maps)[5], const VsParams& p, int grid, cudaStream_t stream) {
+  using C = VsCfg<D>;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e =
+        cudaFuncSetAttribute(vs_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  vs_attn_kernel<D><<<grid, kVsThreads, C::kSmemBytes, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vs_attn(int head_dim, const CUtensorMap (&maps)[5], const VsParams& p, int grid,
+                           cudaStream_t stream) {
+  if (head_dim == 128) return vs_launch_one<128>(maps, p, grid, stream);
+  if (head_dim == 64) return vs_launch_one<64>(maps, p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace spk
