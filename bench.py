@@ -40,7 +40,7 @@ import workloads as W  # noqa: E402
 METRIC = "KV-head-tokens scored+selected+compacted/s at 64K ctx"
 SUITE = ("llama3.1-8b_speckv_16k", "qwen2.5-32b_speckv_64k", "qwen2.5-32b_speckv_64k@1024",
          "qwen2.5-32b_speckv_64k@2048", "qwen2.5-32b_speckv_64k+prefill", "qwen2.5-0.5b_specpc_32k",
-         "cascade_specpc_speckv_128k", "qwen2.5-32b_decode_compressed")
+         "cascade_specpc_speckv_128k", "qwen2.5-32b_decode_compressed", "llama3.1-8b_vs_prefill_16k")
 
 
 def parse(argv=None):
@@ -49,7 +49,9 @@ def parse(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--config", default=W.QWEN32B_64K.name, choices=list(W.CONFIGS))
+    ap.add_argument("--config", default=W.QWEN32B_64K.name,
+                    help="workload name (see workloads.CONFIGS), optionally with @C_max or +prefill")
+    ap.add_argument("--layers", type=int, default=None, help="override the workload's layer count (small captures)")
     ap.add_argument("--cmax", type=int, default=None)
     ap.add_argument("--suite", action="store_true", help="one line per workload (headline included)")
     ap.add_argument("--seed", type=int, default=0)
@@ -61,16 +63,21 @@ def parse(argv=None):
     return ap.parse_args(argv)
 
 
-def config_of(name, cmax=None):
+def config_of(name, cmax=None, layers=None):
     """A workload by name; "<name>@C" sets C_max, "<name>+prefill" runs the
-    scoring after the prefill attention of the window and lookahead rows."""
+    scoring after the prefill attention of the window and lookahead rows;
+    layers overrides the layer count (small profiling captures)."""
     name = name.replace("+prefill", "")
     if "@" in name:
         name, c = name.split("@")
         cmax = int(c)
+    if name not in W.CONFIGS:
+        raise SystemExit(f"unknown workload {name!r}; one of {sorted(W.CONFIGS)}")
     cfg = W.CONFIGS[name]
     if cmax is not None and isinstance(cfg, W.SpecKVConfig):
         cfg = dataclasses.replace(cfg, c_max=cmax)
+    if layers is not None and hasattr(cfg, "layers"):
+        cfg = dataclasses.replace(cfg, layers=layers)
     return cfg
 
 
@@ -678,6 +685,83 @@ def run_decode(args, cfg, P, dev):
     }
 
 
+# ----------------------------------------------------------------- Vertical-Slash sparse prefill
+def vs_tile_work(cfg, vert, sl):
+    """Key tiles the kernel processes (slash tiles + vertical tiles, summed over
+    items) and the (row, key) pairs the pattern makes visible, from the same
+    definitions the kernel and the oracle use."""
+    import torch
+    n, nq = cfg.n, cfg.n_q
+    vert_c, sl_c = vert.cpu().numpy(), sl.cpu().numpy()
+    tiles = 0
+    visible = 0
+    pos = np.arange(n - nq, n)
+    for u in range(cfg.units):
+        S = np.union1d(sl_c[u], [0])
+        V = vert_c[u]
+        for rb in range((nq + 127) // 128):
+            p0 = n - nq + rb * 128
+            p_last = n - nq + min(rb * 128 + 127, nq - 1)
+            t = np.arange(p_last // 128 + 1)
+            lo, hi = p0 - 128 * t - 127, p_last - 128 * t
+            idx = np.searchsorted(S, lo)
+            hit = (idx < S.size) & (S[np.minimum(idx, S.size - 1)] <= hi)
+            cv = np.searchsorted(V, p_last, side="right")
+            tiles += int(hit.sum()) + (cv + 127) // 128
+        # visible pairs: diagonals of S u {0} within each row's prefix, plus
+        # vertical keys not on those diagonals
+        diag = sum(int(np.clip(pos - o + 1, 0, None).astype(bool).sum()) for o in S)
+        vv = sum(int(((V <= p) & ~np.isin(p - V, S)).sum()) for p in pos[:: max(1, nq // 64)]) * max(1, nq // 64)
+        visible += diag + vv
+    return tiles * cfg.g, visible * cfg.g
+
+
+def run_vs(args, cfg, P, dev):
+    """Vertical-Slash sparse prefill over every query row of the sequence,
+    one GPU: the vertical rows' gather (kv_compact) and the sparse attention."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    gen = torch.Generator(device=dev).manual_seed(args.seed)
+    shape_q = (cfg.batch, cfg.layers, cfg.hq, cfg.n_q, cfg.head_dim)
+    shape_k = (cfg.batch, cfg.layers, cfg.hkv, cfg.n, cfg.head_dim)
+    q = (torch.randn(shape_q, generator=gen, device=dev) / cfg.head_dim ** 0.5).to(torch.bfloat16)
+    k = torch.randn(shape_k, generator=gen, device=dev).to(torch.bfloat16)
+    v = torch.randn(shape_k, generator=gen, device=dev).to(torch.bfloat16)
+    vert, sl = W.vs_pattern(cfg, seed=args.seed, device=dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(P.vs_workspace_size(P.binding.vs_shape(q, k, cfg.n_vertical, cfg.n_slash)), dtype=torch.uint8,
+                     device=dev)
+    launches = [("vs_sparse_attention", lambda: P.vs_sparse_attention(q, k, v, vert, sl, out=out, workspace=ws,
+                                                                      stream=stream))]
+    total, per, med, clocks = timed_steps(launches, args.steps, args.warmup, stream)
+    check_device(P, "in the timed steps")
+    ms = total / args.steps
+    tiles, visible = vs_tile_work(cfg, vert, sl)
+    peaks = load_peaks()
+    peak, src = tensor_peak(peaks)
+    tile_flops = tiles * 2 * 2 * 128 * 128 * cfg.head_dim
+    useful_flops = visible * 2 * 2 * cfg.head_dim
+    dense = cfg.batch * cfg.layers * cfg.hq * sum(range(cfg.n - cfg.n_q + 1, cfg.n + 1)) * 2 * 2 * cfg.head_dim
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    achieved = tile_flops / (ms * 1e-3) / 1e12
+    return {
+        "metric": "query rows attended/s (Vertical-Slash sparse prefill)",
+        "value": cfg.batch * cfg.layers * cfg.hq * cfg.n_q / (ms * 1e-3), "unit": "query-head rows/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_median": med,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "n": cfg.n, "n_q": cfg.n_q, "n_vertical": cfg.n_vertical,
+                   "n_slash": cfg.n_slash, "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "tensor", "kernel": "vs_attn_kernel (+ vertical gather)", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": src,
+                     "flops": "executed 128-key tiles x 2 products; useful (visible pairs) and dense-causal "
+                              "figures beside it",
+                     "useful_tflops": useful_flops / (ms * 1e-3) / 1e12,
+                     "density_vs_dense_causal": useful_flops / dense},
+        "gpu_launches": 2 * args.steps, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+    }
+
+
 # ----------------------------------------------------------------- traffic bookkeeping
 # The files that define the scoring kernels and how they are launched.
 SCORING_SOURCES = ("api.cu", "common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh")
@@ -806,7 +890,7 @@ def run_e2e(args, cfg, P, q, k, v, dev, stream, world, max_over_ranks, barrier):
 # ----------------------------------------------------------------- main
 def main(argv=None):
     args = parse(argv)
-    cfg = config_of(args.config, args.cmax)
+    cfg = config_of(args.config, args.cmax, args.layers)
     if args.impl == "reference":
         if not isinstance(cfg, W.SpecKVConfig):
             print(json.dumps({"impl": "reference", "unavailable":
@@ -834,7 +918,7 @@ def main(argv=None):
     names = SUITE if args.suite else (args.config + (f"@{args.cmax}" if args.cmax else ""),)
     lines = []
     for name in names:
-        c = config_of(name)
+        c = config_of(name, layers=None if args.suite else args.layers)
         prefill = name.endswith("+prefill")
         headline = (c == W.QWEN32B_64K) and not prefill
         if isinstance(c, W.SpecKVConfig):
@@ -843,6 +927,8 @@ def main(argv=None):
             continue                         # the other workloads are single-GPU lines
         elif isinstance(c, W.DecodeConfig):
             line = run_decode(args, c, P, dev)
+        elif isinstance(c, W.VSConfig):
+            line = run_vs(args, c, P, dev)
         else:
             line = run_specpc_like(args, c, P, dev)
         lines.append((headline, line))

@@ -48,6 +48,31 @@ def test_suite_names_resolve():
         cfg = bench.config_of(name)
         assert cfg is not None
     assert bench.config_of("qwen2.5-32b_speckv_64k@2048").c_max == 2048
+    assert bench.config_of("qwen2.5-32b_speckv_64k+prefill", layers=2).layers == 2
+
+
+def test_vs_tile_count_matches_a_direct_walk():
+    # the bench's count of processed key tiles equals a plain per-tile check
+    # of "some offset of S u {0} hits the tile" plus the vertical tiles
+    import dataclasses
+    import numpy as np
+    import workloads as W
+    cfg = dataclasses.replace(W.VS_LLAMA8B_16K, layers=1, hkv=2, hq=4, n=1000, n_q=700, n_vertical=50,
+                              n_local=8, n_far=5)
+    vert, sl = W.vs_pattern(cfg, seed=3)
+    tiles, _ = bench.vs_tile_work(cfg, vert, sl)
+    ref = 0
+    for u in range(cfg.units):
+        S = set(sl[u].tolist()) | {0}
+        V = vert[u].numpy()
+        for rb in range((cfg.n_q + 127) // 128):
+            p0 = cfg.n - cfg.n_q + rb * 128
+            pl = cfg.n - cfg.n_q + min(rb * 128 + 127, cfg.n_q - 1)
+            for t in range(pl // 128 + 1):
+                if any(p0 - 128 * t - 127 <= o <= pl - 128 * t for o in S):
+                    ref += 1
+            ref += (int((V <= pl).sum()) + 127) // 128
+    assert tiles == ref * cfg.g
 
 
 def test_cpu_baselines_on_tiny_workloads():

@@ -25,7 +25,7 @@ __all__ = [
     "SpecKVConfig", "SpecPCConfig", "CascadeConfig", "CONFIGS",
     "bf16_round", "bf16_bits", "bf16_decode",
     "tiny_speckv_numpy", "heavy_positions", "speckv_inputs", "specpc_inputs",
-    "specpc_row_weights", "speckv_unit_numpy", "specpc_layer_numpy",
+    "specpc_row_weights", "speckv_unit_numpy", "specpc_layer_numpy", "VSConfig", "vs_pattern",
 ]
 
 
@@ -150,6 +150,38 @@ class DecodeConfig:
         return self.batch * self.layers * self.hkv
 
 
+@dataclasses.dataclass(frozen=True)
+class VSConfig:
+    """Vertical-Slash sparse prefill over an n-token sequence (section
+    "损失函数 / 训练策略": SpecKV's target prefill is Vertical-Slash sparse).
+    Query rows are the last n_q positions; per unit (batch, layer, KV head) the
+    pattern has n_vertical key columns (the sink and random keys) and
+    n_local + n_far diagonals (offsets 0 .. n_local-1 and random far ones)."""
+    name: str
+    batch: int
+    layers: int
+    hq: int
+    hkv: int
+    head_dim: int
+    n: int
+    n_q: int
+    n_vertical: int
+    n_local: int
+    n_far: int
+
+    @property
+    def g(self) -> int:
+        return self.hq // self.hkv
+
+    @property
+    def units(self) -> int:
+        return self.batch * self.layers * self.hkv
+
+    @property
+    def n_slash(self) -> int:
+        return self.n_local + self.n_far
+
+
 TINY = SpecKVConfig("tiny_speckv", batch=1, layers=1, hq=4, hkv=2, head_dim=64,
                     n_in=512, n_window=16, n_lookahead=16, c_max=64, pool=7)
 LLAMA8B_16K = SpecKVConfig("llama3.1-8b_speckv_16k", batch=1, layers=32, hq=32, hkv=8,
@@ -172,8 +204,11 @@ CASCADE_128K = CascadeConfig(
 DECODE_QWEN32B = DecodeConfig("qwen2.5-32b_decode_compressed", batch=1, layers=64, hq=40, hkv=8,
                               head_dim=128, n_kv=320, n_kv_full=65536)
 
+VS_LLAMA8B_16K = VSConfig("llama3.1-8b_vs_prefill_16k", batch=1, layers=32, hq=32, hkv=8, head_dim=128,
+                          n=16384, n_q=16384, n_vertical=1024, n_local=64, n_far=16)
+
 CONFIGS = {c.name: c for c in (TINY, LLAMA8B_16K, QWEN32B_64K, QWEN05B_SPECPC_32K, CASCADE_128K,
-                               DECODE_QWEN32B)}
+                               DECODE_QWEN32B, VS_LLAMA8B_16K)}
 
 
 # ---------------------------------------------------------------------------
@@ -374,3 +409,20 @@ def specpc_layer_numpy(cfg: SpecPCConfig, seed: int, b: int, layer: int):
     q += cfg.q_offset * np.repeat(u, cfg.g, axis=0)[:, None, :]
     q *= np.float32(1.0 / math.sqrt(d))
     return bf16_bits(q), bf16_bits(k)
+
+
+def vs_pattern(cfg: VSConfig, seed: int = 0, device="cpu"):
+    """Seeded Vertical-Slash pattern per unit: vertical = key 0 plus random
+    distinct keys, slash = offsets 0 .. n_local-1 plus random distinct far
+    offsets; both ascending int32 [units, count]."""
+    torch = _torch()
+    rng = np.random.default_rng(seed)
+    vert = np.zeros((cfg.units, cfg.n_vertical), np.int32)
+    sl = np.zeros((cfg.units, cfg.n_slash), np.int32)
+    for u in range(cfg.units):
+        if cfg.n_vertical:
+            v = rng.choice(np.arange(1, cfg.n), size=cfg.n_vertical - 1, replace=False)
+            vert[u] = np.sort(np.concatenate([[0], v]))
+        far = rng.choice(np.arange(cfg.n_local, cfg.n), size=cfg.n_far, replace=False)
+        sl[u] = np.sort(np.concatenate([np.arange(cfg.n_local), far]))
+    return torch.from_numpy(vert).to(device), torch.from_numpy(sl).to(device)
