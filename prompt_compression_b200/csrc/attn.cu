@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "score.cuh"
 
 namespace spk {
@@ -47,6 +48,7 @@ constexpr int kAttnProducerWarp = 4;
 constexpr int kAttnMmaWarp = 5;
 constexpr int kAttnThreads = 6 * 32;
 constexpr float kRescaleLog2 = 8.f;    // lazy rescale threshold (P <= 2^8)
+constexpr int kAttnPolyOf8 = 2;        // exponential pairs (of 8) evaluated on the FMA pipe
 
 template <int D>
 struct AttnCfg {
@@ -86,10 +88,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// (lo, hi) -> bf16x2 with lo in the low half: one packed conversion.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return a | (b << 16);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Row r (0..127) of a row-offset block: v split into three bf16 terms
@@ -346,17 +348,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         // P = 2^(c2 s - m) (masked keys: 2^-inf = 0), packed as bf16 pairs
-        float sum0 = 0.f, sum1 = 0.f;
+        // packed fp32x2 math; 2 of every 8 exponential pairs on the FMA pipe
+        // (exp2_poly.cuh), the rest on the MUFU
+        const float2 c2v = f2(p.c2, p.c2), nm = f2(-m, -m);
+        float2 acc2 = f2(0.f, 0.f);
         uint32_t pk[64];
 #pragma unroll
         for (int k = 0; k < 64; ++k) {
-          const float e0 = ex2_approx(fmaf(s[2 * k], p.c2, -m));
-          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.c2, -m));
-          sum0 += e0;
-          sum1 += e1;
-          pk[k] = pack_bf16(e0, e1);
+          const float2 tt = __ffma2_rn(f2(s[2 * k], s[2 * k + 1]), c2v, nm);
+          const float2 e = ((k & 7) < kAttnPolyOf8) ? exp2_fma_pair(tt) : exp2_mufu_pair(tt);
+          acc2 = __fadd2_rn(acc2, e);
+          pk[k] = pack_bf16(e.x, e.y);
         }
-        l += sum0 + sum1;
+        l += acc2.x + acc2.y;
         {
           uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
           uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);

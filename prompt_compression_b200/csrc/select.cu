@@ -377,16 +377,26 @@ __global__ void __launch_bounds__(kSelThreads, 4)
   for (int b = tid; b < kBins; b += kSelThreads) sh.hist[b] = 0;
   if (tid == 0) { sh.n_a = 0; sh.n_b = 0; }
   __syncthreads();
+  // Histogram adds are run-length aggregated per thread: the pooled values
+  // crowd into a few bins, and contended shared-memory atomics on the same
+  // bin serialize, so a thread adds a bin's count once per run of equal bins.
+  uint32_t run_bin = kBins, run_cnt = 0;
   pooled_sweep(s, n, pool_r, pool_mode, sh.tile, [&](int j, bool valid, float p) {
-    uint32_t bin = kBins;
-    if (valid) {
-      if (pout) pout[j] = p;
-      const uint32_t key = float_key(p);
-      if (select) keys[j] = key;
-      bin = key >> 20;
+    if (!valid) return;
+    if (pout) pout[j] = p;
+    if (!select) return;
+    const uint32_t key = float_key(p);
+    keys[j] = key;
+    const uint32_t bin = key >> 20;
+    if (bin == run_bin) {
+      ++run_cnt;
+    } else {
+      if (run_cnt) atomicAdd(&sh.hist[run_bin], run_cnt);
+      run_bin = bin;
+      run_cnt = 1;
     }
-    if (select) hist_add(sh.hist, bin);
   });
+  if (run_cnt) atomicAdd(&sh.hist[run_bin], run_cnt);
   if (C == 0) return;
   if (C >= n) {
     for (int j = tid; j < n; j += kSelThreads) out[j] = j;

@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "score.cuh"
 
 namespace spk {
@@ -43,6 +44,7 @@ constexpr int kVsProducerWarp = 4;
 constexpr int kVsMmaWarp = 5;
 constexpr int kVsThreads = 6 * 32;
 constexpr float kVsRescale = 8.f;
+constexpr int kVsPolyOf8 = 2;          // exponential pairs (of 8) evaluated on the FMA pipe
 
 template <int D>
 struct VsCfg {
@@ -76,10 +78,10 @@ __device__ __forceinline__ void vs_tmem_st32(uint32_t taddr, const uint32_t (&r)
       : "memory");
 }
 
+// (lo, hi) -> bf16x2 with lo in the low half: one packed conversion.
 __device__ __forceinline__ uint32_t vs_pack_bf16(float lo, float hi) {
-  const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return a | (b << 16);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __device__ __forceinline__ int vs_site(int role, int which) { return 400 + role * 10 + which; }
@@ -472,18 +474,21 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         }
         // P = 2^(c2 s - m): masked keys (s = -inf) give 0; a row that has
         // seen no key yet (m = -inf) has only masked keys here
+        // (the FMA-pipe exponential turns a masked key into 2^-126 instead of
+        // 0: far below the rounding of the sum and of O, and wiped by the
+        // rescale when a row sees its first key)
         const float mm = m == -INFINITY ? 0.f : m;
-        float sum0 = 0.f, sum1 = 0.f;
+        const float2 c2v = f2(p.c2, p.c2), nm = f2(-mm, -mm);
+        float2 acc2 = f2(0.f, 0.f);
         uint32_t pk[64];
 #pragma unroll
         for (int k = 0; k < 64; ++k) {
-          const float e0 = ex2_approx(fmaf(s[2 * k], p.c2, -mm));
-          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.c2, -mm));
-          sum0 += e0;
-          sum1 += e1;
-          pk[k] = vs_pack_bf16(e0, e1);
+          const float2 tt = __ffma2_rn(f2(s[2 * k], s[2 * k + 1]), c2v, nm);
+          const float2 e = ((k & 7) < kVsPolyOf8) ? exp2_fma_pair(tt) : exp2_mufu_pair(tt);
+          acc2 = __fadd2_rn(acc2, e);
+          pk[k] = vs_pack_bf16(e.x, e.y);
         }
-        l += sum0 + sum1;
+        l += acc2.x + acc2.y;
         {
           uint32_t (&p0r)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
           uint32_t (&p1r)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);

@@ -103,7 +103,7 @@ def test_vs_attention_full_pattern_is_dense(P):
     sl = np.zeros((1, 0), np.int32)
     _check(P, qb, kb, vb, vert, sl)
     out, _ = _run(P, qb, kb, vb, vert, sl)
-    ref, _ = oracle.prefill_unit(qb[0, 0], kb[0, 0], vb[0, 0], 300, 0, 300)
+    ref, _ = oracle.prefill_unit(qb[0, 0], kb[0, 0, 0], vb[0, 0, 0], 300, 0, 300)
     assert np.abs(W.bf16_decode(bits_of(out))[0, 0] - ref).max() <= 2.0 ** -8 * np.abs(W.bf16_decode(vb)).max()
 
 
