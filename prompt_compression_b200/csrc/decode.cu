@@ -25,12 +25,17 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "exp2_poly.cuh"
 #include "score.cuh"
 
 namespace spk {
 namespace {
 
-constexpr int kDecMaxWarps = 16;
+// Up to 12 warps; groups of up to 6 query heads fit 80 registers, so two
+// CTAs (one unit each) share an SM; larger groups keep one CTA per SM.
+constexpr int kDecMaxWarps = 12;
+template <int G>
+constexpr int dec_blocks_per_sm() { return G <= 6 ? 2 : 1; }
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
@@ -68,7 +73,7 @@ __device__ __forceinline__ void unpack(const typename RowSlice<D>::T& r, float (
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecMaxWarps * 32)
+__global__ void __launch_bounds__(kDecMaxWarps * 32, dec_blocks_per_sm<G>())
     decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
                   float* __restrict__ out, int n_kv, float c2) {
   using S = RowSlice<D>;
@@ -109,33 +114,38 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32)
     }
     const int t = t0 + lane;
     const bool valid = t < n_kv;
-    // logits of this lane's row for every query head of the group
+    // logits of this lane's row for every query head of the group: the K
+    // row in two halves (D/16 16-byte pieces in flight at once), packed
+    // fp32x2 multiply-adds
     const uint4* krow = reinterpret_cast<const uint4*>(kr + static_cast<size_t>(valid ? t : t0) * D);
-    float z[G];
+    float2 z2[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) z[h] = 0.f;
-    uint4 kbuf[D / 8];   // the whole row in flight at once
+    for (int h = 0; h < G; ++h) z2[h] = f2(0.f, 0.f);
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) kbuf[c] = __ldg(krow + c);
+    for (int half = 0; half < 2; ++half) {
+      uint4 kbuf[D / 16];
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 kk = kbuf[c];
-      const float kf[8] = {bf16_lo(kk.x), bf16_hi(kk.x), bf16_lo(kk.y), bf16_hi(kk.y),
-                           bf16_lo(kk.z), bf16_hi(kk.z), bf16_lo(kk.w), bf16_hi(kk.w)};
+      for (int c = 0; c < D / 16; ++c) kbuf[c] = __ldg(krow + half * (D / 16) + c);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4 qa = *reinterpret_cast<const float4*>(&q_s[h][c * 8]);
-        const float4 qb = *reinterpret_cast<const float4*>(&q_s[h][c * 8 + 4]);
-        z[h] = fmaf(qa.x, kf[0], z[h]);
-        z[h] = fmaf(qa.y, kf[1], z[h]);
-        z[h] = fmaf(qa.z, kf[2], z[h]);
-        z[h] = fmaf(qa.w, kf[3], z[h]);
-        z[h] = fmaf(qb.x, kf[4], z[h]);
-        z[h] = fmaf(qb.y, kf[5], z[h]);
-        z[h] = fmaf(qb.z, kf[6], z[h]);
-        z[h] = fmaf(qb.w, kf[7], z[h]);
+      for (int c = 0; c < D / 16; ++c) {
+        const uint4 kk = kbuf[c];
+        const float2 k0 = f2(bf16_lo(kk.x), bf16_hi(kk.x)), k1 = f2(bf16_lo(kk.y), bf16_hi(kk.y));
+        const float2 k2 = f2(bf16_lo(kk.z), bf16_hi(kk.z)), k3 = f2(bf16_lo(kk.w), bf16_hi(kk.w));
+        const int e0 = (half * (D / 16) + c) * 8;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float4 qa = *reinterpret_cast<const float4*>(&q_s[h][e0]);
+          const float4 qb = *reinterpret_cast<const float4*>(&q_s[h][e0 + 4]);
+          z2[h] = __ffma2_rn(f2(qa.x, qa.y), k0, z2[h]);
+          z2[h] = __ffma2_rn(f2(qa.z, qa.w), k1, z2[h]);
+          z2[h] = __ffma2_rn(f2(qb.x, qb.y), k2, z2[h]);
+          z2[h] = __ffma2_rn(f2(qb.z, qb.w), k3, z2[h]);
+        }
       }
     }
+    float z[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) z[h] = z2[h].x + z2[h].y;
     // online softmax over the block, per query head
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -167,7 +177,11 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32)
       for (int h = 0; h < G; ++h) {
         const float pj = p_s[warp][h][j];
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[h][e] = fmaf(pj, vf[e], acc[h][e]);
+        for (int e = 0; e < E; e += 2) {
+          const float2 a = __ffma2_rn(f2(pj, pj), f2(vf[e], vf[e + 1]), f2(acc[h][e], acc[h][e + 1]));
+          acc[h][e] = a.x;
+          acc[h][e + 1] = a.y;
+        }
       }
     }
     __syncwarp();   // the buffer and p_s are free for the next block

@@ -9,24 +9,21 @@
 // One CTA (512 threads) per row of candidates.  Pooled values are turned into
 // order-preserving 32-bit keys (a larger float gives a larger key).
 //   1. sweep 1: tiles of 2048 scores plus the pooling halo are staged in
-//      shared memory (five independent loads per thread in flight); every
-//      pooled value is formed there and counted in a 4096-bin histogram of
-//      its key's top 12 bits.  The bin B1 that holds the C-th largest key
-//      follows from one scan of the histogram.
-//   2. sweep 2 forms the same pooled values again (the same fp32 operations,
-//      so the same keys): keys in bins above B1 are selected outright and
-//      their indices collected; keys in B1 are collected with their index as
-//      candidates.  Both lists live in shared memory.
-//   3. the candidates are sorted by (key descending, index ascending), the
-//      first C - |selected| of them complete the selection, and the C indices
-//      are sorted ascending: ties go to the lower index, the output is
-//      ordered, and the result does not depend on the order in which threads
-//      appended to the lists.
-// When C exceeds 2048, or more than 2048 candidates share bin B1 (long runs of
-// equal values), a general path takes over: the keys go to the workspace and
-// a three-level radix select (12 + 12 + 8 bits) finds the exact C-th key T;
-// an ordered ballot walk over each warp's contiguous share of the row emits
-// the indices ascending, keys equal to T lowest index first.
+//      shared memory (five independent loads per thread, the next tile's
+//      issued before the current one is pooled); every pooled value is
+//      formed there, its key written to the workspace (rows padded to 16
+//      bytes) and its top 12 bits counted in a 4096-bin histogram
+//      (run-length aggregated per thread: the values crowd into few bins).
+//   2. the exact key T of the C-th largest, and how many keys equal to T to
+//      take, from two more histograms (the next 12, then the last 8 bits) of
+//      only the keys that match the prefix found so far; the workspace keys
+//      are swept with 16-byte loads, four in flight per thread.
+//   3. ordered emission: each warp owns a contiguous share of the row; one
+//      walk counts its keys above and equal to T, a CTA prefix gives every
+//      warp its output offset and its share of the ties (lowest index
+//      first), a second walk writes the indices in ascending order.
+// No sort and no shared-memory list: any k, deterministic, ties to the
+// lower index.
 #include "common.cuh"
 #include "score.cuh"
 
@@ -39,7 +36,6 @@ constexpr int kBins = 4096;
 constexpr int kTile = 2048;                 // candidates per staged tile
 constexpr int kHaloMax = 256;               // pooling radius served from the staged tile
 constexpr int kTileLoads = (kTile + 2 * kHaloMax + kSelThreads - 1) / kSelThreads;   // 5
-constexpr int kListMax = 2048;              // shared-memory selection lists
 
 // Monotone map from finite floats to uint32 (larger float -> larger key);
 // -0 is folded onto +0 so that the two compare equal, as they do as floats.
@@ -196,40 +192,11 @@ __device__ __forceinline__ void pooled_sweep(const float* __restrict__ s, int n,
   }
 }
 
-// Ascending bitonic sort of a[0, P) in shared memory, P a power of two.
-template <typename T>
-__device__ __forceinline__ void bitonic_sort(T* a, int P) {
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = threadIdx.x; i < P; i += kSelThreads) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const T x = a[i], y = a[ixj];
-          const bool up = (i & k) == 0;
-          if ((x > y) == up) {
-            a[i] = y;
-            a[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-}
-
-__device__ __forceinline__ int pow2_at_least(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
 struct SelShared {
   float tile[kTile + 2 * kHaloMax];
   uint32_t hist[kBins];
-  unsigned long long cand[kListMax];   // (~key << 32) | index: ascending = key desc, index asc
-  int list[kListMax];
   int warp_tot[33];
-  int s_bin, s_rem, n_a, n_b;
+  int s_bin, s_rem;
 };
 
 // Calls f(j, valid, key_j) for every key of the row (keys padded to a
@@ -257,106 +224,106 @@ __device__ __forceinline__ void key_sweep(const uint32_t* __restrict__ keys, int
   }
 }
 
-// Warp-aggregated append of the lanes with pred to a shared list: returns
-// the lane's slot (or -1), one atomic per warp.
-__device__ __forceinline__ int warp_append(int* counter, bool pred) {
-  const uint32_t m = __ballot_sync(0xffffffffu, pred);
-  const int lane = threadIdx.x & 31;
-  int base = 0;
-  if (lane == 0 && m) base = atomicAdd(counter, __popc(m));
-  base = __shfl_sync(0xffffffffu, base, 0);
-  return pred ? base + __popc(m & ((1u << lane) - 1u)) : -1;
+// Histogram of the keys that match `prefix` on their top `known` bits, by
+// their next `width` bits (plain atomics: these keys spread over the bins).
+__device__ __forceinline__ void prefix_hist(SelShared& sh, const uint32_t* __restrict__ keys, int n, uint32_t prefix,
+                                            int known, int width) {
+  const int nb = 1 << width;
+  for (int b = threadIdx.x; b < nb; b += kSelThreads) sh.hist[b] = 0;
+  __syncthreads();
+  const int shift = 32 - known - width;
+  key_sweep(keys, n, [&](int, bool valid, uint32_t key) {
+    if (valid && (key >> (32 - known)) == prefix) atomicAdd(&sh.hist[(key >> shift) & (nb - 1)], 1u);
+  });
+  __syncthreads();
 }
 
-// General path (C > kListMax, or more than kListMax keys share even a 24-bit
-// prefix with the C-th largest): three radix levels over the keys in the
-// workspace, then an ordered ballot emission.
-__device__ __noinline__ void select_general(SelShared& sh, int n, int C, const uint32_t* __restrict__ keys,
-                                            int* __restrict__ out) {
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  uint32_t* hist = sh.hist;
-  __syncthreads();
-  for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0;
-  __syncthreads();
-  key_sweep(keys, n, [&](int, bool valid, uint32_t key) { hist_add(hist, valid ? key >> 20 : kBins); });
-  __syncthreads();
-  find_bin(hist, kBins, C, sh.warp_tot, &sh.s_bin, &sh.s_rem);
-  uint32_t prefix = static_cast<uint32_t>(sh.s_bin);        // top 12 bits of T
-  int remaining = sh.s_rem;
-  for (int b = tid; b < kBins; b += kSelThreads) hist[b] = 0;
-  __syncthreads();
-  key_sweep(keys, n, [&](int, bool valid, uint32_t key) {
-    hist_add(hist, valid && (key >> 20) == prefix ? (key >> 8) & 4095u : kBins);
-  });
-  __syncthreads();
-  find_bin(hist, kBins, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
-  prefix = (prefix << 12) | static_cast<uint32_t>(sh.s_bin);   // top 24 bits of T
-  remaining = sh.s_rem;
-  for (int b = tid; b < 256; b += kSelThreads) hist[b] = 0;
-  __syncthreads();
-  key_sweep(keys, n, [&](int, bool valid, uint32_t key) {
-    hist_add(hist, valid && (key >> 8) == prefix ? key & 255u : kBins);
-  });
-  __syncthreads();
-  find_bin(hist, 256, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
-  const uint32_t T = (prefix << 8) | static_cast<uint32_t>(sh.s_bin);
-  const int take_eq = sh.s_rem;   // keys equal to T to take, lowest index first
-
-  // ordered emission: warp w owns [w * chunk, (w + 1) * chunk)
-  const int chunk = ((n + kSelWarps - 1) / kSelWarps + 31) & ~31;
-  const int beg = warp * chunk < n ? warp * chunk : n;
-  const int end = beg + chunk < n ? beg + chunk : n;
+// Ordered emission of the selection {key > T} u {the first take_eq keys ==
+// T}: warp w owns a contiguous, 128-key-aligned share of the row; one walk
+// counts its keys above and equal to T, a CTA-wide prefix gives every warp
+// its output offset and its share of the ties, and a second walk writes the
+// indices in ascending order (lane l holds keys 4l .. 4l + 3 of each
+// 128-key step; output positions by warp scans).
+__device__ __forceinline__ void emit_ordered(SelShared& sh, const uint32_t* __restrict__ keys, int n, uint32_t T,
+                                             int take_eq, int* __restrict__ out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int chunk = ((n + kSelWarps - 1) / kSelWarps + 127) & ~127;
+  const int beg = min(warp * chunk, n), end = min(beg + chunk, n);
+  const uint4* kv = reinterpret_cast<const uint4*>(keys);
   int gt = 0, eq = 0;
-  for (int j0 = beg; j0 < end; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < end ? keys[j] : 0u;
-    gt += __popc(__ballot_sync(0xffffffffu, j < end && key > T));
-    eq += __popc(__ballot_sync(0xffffffffu, j < end && key == T));
+  for (int j0 = beg; j0 < end; j0 += 4 * 128) {
+    uint4 w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + q * 128 + 4 * lane;
+      w[q] = j < end ? kv[j >> 2] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + q * 128 + 4 * lane;
+      const uint32_t k4[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool valid = j + e < end;
+        gt += valid && k4[e] > T;
+        eq += valid && k4[e] == T;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
   }
   int total;
   // one value per warp: lane 0 carries it, the others add nothing
   const int eq_before = __shfl_sync(0xffffffffu, block_exclusive_scan(lane == 0 ? eq : 0, sh.warp_tot, total), 0);
-  int my_eq = take_eq - eq_before;
-  my_eq = my_eq < 0 ? 0 : (my_eq > eq ? eq : my_eq);
+  const int my_eq = min(max(take_eq - eq_before, 0), eq);   // ties this warp takes, lowest index first
   int pos = __shfl_sync(0xffffffffu, block_exclusive_scan(lane == 0 ? gt + my_eq : 0, sh.warp_tot, total), 0);
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int j0 = beg; j0 < end; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < end ? keys[j] : 0u;
-    const bool is_eq = j < end && key == T;
-    const uint32_t eq_bal = __ballot_sync(0xffffffffu, is_eq);
-    const bool sel = (j < end && key > T) || (is_eq && static_cast<int>(__popc(eq_bal & lt_mask)) < my_eq);
-    const uint32_t sel_bal = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[pos + __popc(sel_bal & lt_mask)] = j;
-    pos += __popc(sel_bal);
-    my_eq -= __popc(eq_bal);
+  int eq_seen = 0;
+  for (int j0 = beg; j0 < end; j0 += 128) {
+    const int j = j0 + 4 * lane;
+    const uint4 w = j < end ? kv[j >> 2] : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t k4[4] = {w.x, w.y, w.z, w.w};
+    int n_eq = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) n_eq += (j + e < end) && k4[e] == T;
+    int eq_pre = n_eq;                                 // inclusive warp scan of the ties
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, eq_pre, o);
+      if (lane >= o) eq_pre += y;
+    }
+    int rank = eq_seen + eq_pre - n_eq;                // ties before this lane's first
+    bool sel[4];
+    int n_sel = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool valid = j + e < end;
+      const bool is_eq = valid && k4[e] == T;
+      sel[e] = (valid && k4[e] > T) || (is_eq && rank < my_eq);
+      rank += is_eq;
+      n_sel += sel[e];
+    }
+    int sel_pre = n_sel;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, sel_pre, o);
+      if (lane >= o) sel_pre += y;
+    }
+    int at = pos + sel_pre - n_sel;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (sel[e]) out[at++] = j + e;
+    pos += __shfl_sync(0xffffffffu, sel_pre, 31);
+    eq_seen += __shfl_sync(0xffffffffu, eq_pre, 31);
   }
-}
-
-// The candidates (sh.n_b <= kListMax of them) sorted by (key desc, index
-// asc) complete the selected list with `need` entries; the C indices are
-// then sorted ascending and written.
-__device__ __forceinline__ void finish_selection(SelShared& sh, int need, int C, int* __restrict__ out) {
-  const int tid = threadIdx.x;
-  const int n_a = sh.n_a, n_b = sh.n_b;
-  const int pb = pow2_at_least(n_b);
-  for (int t = n_b + tid; t < pb; t += kSelThreads) sh.cand[t] = ~0ull;
-  __syncthreads();
-  bitonic_sort(sh.cand, pb);
-  for (int t = tid; t < need; t += kSelThreads) sh.list[n_a + t] = static_cast<int>(sh.cand[t] & 0xffffffffu);
-  const int pc = pow2_at_least(C);
-  for (int t = C + tid; t < pc; t += kSelThreads) sh.list[t] = 0x7fffffff;
-  __syncthreads();
-  bitonic_sort(sh.list, pc);
-  for (int t = tid; t < C; t += kSelThreads) out[t] = sh.list[t];
 }
 
 __global__ void __launch_bounds__(kSelThreads, 4)
     topk_kernel(const float* __restrict__ scores, int n_cand, int pool_r, int pool_mode, int k, int n_tail,
                 int* __restrict__ idx, float* __restrict__ pooled, uint32_t* __restrict__ keys_ws, int key_stride) {
-  extern __shared__ __align__(16) uint8_t sel_smem[];   // 50 KB: above the 48 KB of static shared memory
-  SelShared& sh = *reinterpret_cast<SelShared*>(sel_smem);
+  __shared__ SelShared sh;
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   const int n = n_cand;
@@ -373,13 +340,12 @@ __global__ void __launch_bounds__(kSelThreads, 4)
   float* pout = pooled ? pooled + static_cast<size_t>(u) * n : nullptr;
   const bool select = C > 0 && C < n;
 
-  // 1. pooled values -> (optional output), keys to the workspace, histogram of their top 12 bits
+  // 1. pooled values -> (optional output), keys to the workspace, histogram
+  // of their top 12 bits.  The adds are run-length aggregated per thread: the
+  // pooled values crowd into a few bins, and contended shared-memory atomics
+  // on one bin serialize.
   for (int b = tid; b < kBins; b += kSelThreads) sh.hist[b] = 0;
-  if (tid == 0) { sh.n_a = 0; sh.n_b = 0; }
   __syncthreads();
-  // Histogram adds are run-length aggregated per thread: the pooled values
-  // crowd into a few bins, and contended shared-memory atomics on the same
-  // bin serialize, so a thread adds a bin's count once per run of equal bins.
   uint32_t run_bin = kBins, run_cnt = 0;
   pooled_sweep(s, n, pool_r, pool_mode, sh.tile, [&](int j, bool valid, float p) {
     if (!valid) return;
@@ -403,51 +369,23 @@ __global__ void __launch_bounds__(kSelThreads, 4)
     return;
   }
   __syncthreads();               // keys and histogram complete
-  if (C > kListMax) {
-    select_general(sh, n, C, keys, out);
-    return;
-  }
+
+  // 2. the exact key T of the C-th largest: 12 + 12 + 8 bits, the later
+  // levels histogramming only the keys that match the prefix so far
   find_bin(sh.hist, kBins, C, sh.warp_tot, &sh.s_bin, &sh.s_rem);
-  const uint32_t b1 = static_cast<uint32_t>(sh.s_bin);
-  const int need1 = sh.s_rem;    // keys of bin b1 still to take (>= 1)
-  for (int b = tid; b < kBins; b += kSelThreads) sh.hist[b] = 0;
-  __syncthreads();
+  uint32_t prefix = static_cast<uint32_t>(sh.s_bin);
+  int remaining = sh.s_rem;
+  prefix_hist(sh, keys, n, prefix, 12, 12);
+  find_bin(sh.hist, kBins, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  prefix = (prefix << 12) | static_cast<uint32_t>(sh.s_bin);
+  remaining = sh.s_rem;
+  prefix_hist(sh, keys, n, prefix, 24, 8);
+  find_bin(sh.hist, 256, remaining, sh.warp_tot, &sh.s_bin, &sh.s_rem);
+  const uint32_t T = (prefix << 8) | static_cast<uint32_t>(sh.s_bin);
+  const int take_eq = sh.s_rem;  // keys equal to T to take, lowest index first
 
-  // 2. bins above b1 are selected; bin b1's keys are candidates, histogrammed on their next 12 bits
-  key_sweep(keys, n, [&](int j, bool valid, uint32_t key) {
-    const uint32_t bin = key >> 20;
-    const bool in_b = valid && bin == b1;
-    if (in_b) atomicAdd(&sh.hist[(key >> 8) & 4095u], 1u);
-    const int pa = warp_append(&sh.n_a, valid && bin > b1);   // fewer than C <= kListMax of these
-    if (pa >= 0) sh.list[pa] = j;
-    const int pb = warp_append(&sh.n_b, in_b);
-    if (pb >= 0 && pb < kListMax) sh.cand[pb] = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(j);
-  });
-  __syncthreads();
-  if (sh.n_b <= kListMax) {
-    finish_selection(sh, need1, C, out);
-    return;
-  }
-
-  // 3. too many candidates: refine bin b1 by the next 12 bits
-  find_bin(sh.hist, kBins, need1, sh.warp_tot, &sh.s_bin, &sh.s_rem);
-  const uint32_t p24 = (b1 << 12) | static_cast<uint32_t>(sh.s_bin);
-  const int need2 = sh.s_rem;
-  if (tid == 0) sh.n_b = 0;
-  __syncthreads();
-  key_sweep(keys, n, [&](int j, bool valid, uint32_t key) {
-    const uint32_t pre = key >> 8;
-    const int pa = warp_append(&sh.n_a, valid && (key >> 20) == b1 && pre > p24);
-    if (pa >= 0) sh.list[pa] = j;
-    const int pb = warp_append(&sh.n_b, valid && pre == p24);
-    if (pb >= 0 && pb < kListMax) sh.cand[pb] = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(j);
-  });
-  __syncthreads();
-  if (sh.n_b <= kListMax) {
-    finish_selection(sh, need2, C, out);
-    return;
-  }
-  select_general(sh, n, C, keys, out);   // long runs of equal values
+  // 3. ordered emission
+  emit_ordered(sh, keys, n, T, take_eq, out);
 }
 
 }  // namespace
@@ -462,16 +400,7 @@ size_t topk_ws_bytes(int units, int n_cand) {
 cudaError_t launch_topk(const float* scores, int units, int n_cand, int pool_mode, int pool_kernel, int k,
                         int n_tail, int* idx, float* pooled, void* ws, cudaStream_t stream) {
   if (units == 0) return cudaSuccess;
-  static thread_local int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(SelShared)));
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
-  topk_kernel<<<units, kSelThreads, sizeof(SelShared), stream>>>(scores, n_cand, pool_kernel / 2, pool_mode, k, n_tail, idx,
+  topk_kernel<<<units, kSelThreads, 0, stream>>>(scores, n_cand, pool_kernel / 2, pool_mode, k, n_tail, idx,
                                                  pooled, static_cast<uint32_t*>(ws), key_stride(n_cand));
   return cudaGetLastError();
 }
