@@ -784,8 +784,8 @@ def run_vs(args, cfg, P, dev):
 
 
 # ----------------------------------------------------------------- traffic bookkeeping
-# The files that define the scoring kernels and how they are launched.
-SCORING_SOURCES = ("api.cu", "common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh")
+# The files that define the scoring kernels (device code and their parameter block).
+SCORING_SOURCES = ("common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh")
 
 
 def kernel_source_digest():

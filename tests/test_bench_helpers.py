@@ -36,6 +36,7 @@ def test_digest_covers_the_scoring_sources_only():
     a = bench.kernel_source_digest()
     assert len(a) == 64 and a == bench.kernel_source_digest()
     assert "decode.cu" not in bench.SCORING_SOURCES and "score.cu" in bench.SCORING_SOURCES
+    assert "api.cu" not in bench.SCORING_SOURCES
 
 
 def test_exp2_peak_from_unit_counts():
