@@ -31,11 +31,14 @@
 namespace spk {
 namespace {
 
-// Up to 12 warps; groups of up to 6 query heads fit 80 registers, so two
-// CTAs (one unit each) share an SM; larger groups keep one CTA per SM.
+// Up to 12 warps.  A short cache (at most one 32-row block per warp) reads
+// each K row in two halves, so that groups of up to 6 query heads fit 80
+// registers and two CTAs (one unit each) share an SM; a long cache (many
+// blocks per warp, where the exposed latency of the second half would
+// repeat block after block) keeps the whole row in flight, one CTA per SM.
 constexpr int kDecMaxWarps = 12;
-template <int G>
-constexpr int dec_blocks_per_sm() { return G <= 6 ? 2 : 1; }
+template <int G, bool LONG>
+constexpr int dec_blocks_per_sm() { return (G <= 6 && !LONG) ? 2 : 1; }
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
@@ -72,8 +75,8 @@ __device__ __forceinline__ void unpack(const typename RowSlice<D>::T& r, float (
   }
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(kDecMaxWarps * 32, dec_blocks_per_sm<G>())
+template <int D, int G, bool LONG>
+__global__ void __launch_bounds__(kDecMaxWarps * 32, dec_blocks_per_sm<G, LONG>())
     decode_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
                   float* __restrict__ out, int n_kv, float c2) {
   using S = RowSlice<D>;
@@ -121,17 +124,19 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, dec_blocks_per_sm<G>())
     float2 z2[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) z2[h] = f2(0.f, 0.f);
+    constexpr int kParts = LONG ? 1 : 2;               // pieces of the row in flight at once
+    constexpr int kPer = D / 8 / kParts;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint4 kbuf[D / 16];
+    for (int half = 0; half < kParts; ++half) {
+      uint4 kbuf[kPer];
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) kbuf[c] = __ldg(krow + half * (D / 16) + c);
+      for (int c = 0; c < kPer; ++c) kbuf[c] = __ldg(krow + half * kPer + c);
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
+      for (int c = 0; c < kPer; ++c) {
         const uint4 kk = kbuf[c];
         const float2 k0 = f2(bf16_lo(kk.x), bf16_hi(kk.x)), k1 = f2(bf16_lo(kk.y), bf16_hi(kk.y));
         const float2 k2 = f2(bf16_lo(kk.z), bf16_hi(kk.z)), k3 = f2(bf16_lo(kk.w), bf16_hi(kk.w));
-        const int e0 = (half * (D / 16) + c) * 8;
+        const int e0 = (half * kPer + c) * 8;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float4 qa = *reinterpret_cast<const float4*>(&q_s[h][e0]);
@@ -214,27 +219,33 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, dec_blocks_per_sm<G>())
   }
 }
 
-template <int D, int G>
-cudaError_t launch_g(const void* q, const void* k, const void* v, float* out, int units, int n_kv, float c2,
-                     cudaStream_t stream) {
-  // one warp per 32-row block, up to 16; each warp's V block in shared memory
-  int warps = (n_kv + 31) / 32;
-  warps = warps < 1 ? 1 : (warps > kDecMaxWarps ? kDecMaxWarps : warps);
-  const int smem = warps * 32 * D * 2;
-  static_assert(32 * D * 2 >= G * D * 4, "a warp's V buffer holds its merge state");
+template <int D, int G, bool LONG>
+cudaError_t launch_gl(const void* q, const void* k, const void* v, float* out, int units, int n_kv, float c2,
+                      int warps, cudaStream_t stream) {
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, LONG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kDecMaxWarps * 32 * D * 2);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  decode_kernel<D, G><<<units, warps * 32, smem, stream>>>(static_cast<const uint16_t*>(q),
-                                                           static_cast<const uint16_t*>(k),
-                                                           static_cast<const uint16_t*>(v), out, n_kv, c2);
+  decode_kernel<D, G, LONG><<<units, warps * 32, warps * 32 * D * 2, stream>>>(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), static_cast<const uint16_t*>(v), out, n_kv,
+      c2);
   return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_g(const void* q, const void* k, const void* v, float* out, int units, int n_kv, float c2,
+                     cudaStream_t stream) {
+  // one warp per 32-row block, up to 12; each warp's V block in shared memory
+  static_assert(32 * D * 2 >= G * D * 4, "a warp's V buffer holds its merge state");
+  const int blocks = (n_kv + 31) / 32;
+  const int warps = blocks < 1 ? 1 : (blocks > kDecMaxWarps ? kDecMaxWarps : blocks);
+  if (blocks <= kDecMaxWarps) return launch_gl<D, G, false>(q, k, v, out, units, n_kv, c2, warps, stream);
+  return launch_gl<D, G, true>(q, k, v, out, units, n_kv, c2, warps, stream);
 }
 
 template <int D>
