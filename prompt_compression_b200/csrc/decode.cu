@@ -40,12 +40,6 @@ constexpr int kDecMaxWarps = 12;
 template <int G, bool LONG>
 constexpr int dec_blocks_per_sm() { return (G <= 6 && !LONG) ? 2 : 1; }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 template <int D>
 struct RowSlice;   // one lane's d/32 bf16 elements of a row
 template <>
@@ -170,7 +164,7 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, dec_blocks_per_sm<G, LONG>(
       for (int e = 0; e < E; ++e) acc[h][e] *= alpha;
       p_s[warp][h][lane] = pz;
     }
-    cp_async_wait_all();
+    cp_async_wait<0>();
     __syncwarp();
     // weighted V sum over the block's rows (from shared memory); lane owns E elements of a row
     const typename S::T* vs = reinterpret_cast<const typename S::T*>(vbuf);

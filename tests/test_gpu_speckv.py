@@ -210,17 +210,18 @@ def test_topk_select_direct(P):
 
 @pytest.mark.parametrize("mode", ["max", "avg"])
 def test_topk_paths_on_continuous_scores(P, mode):
-    """Both selection paths on continuous scores: the shared-memory path (C up
-    to 2048 with few candidates in the threshold bin) and the general radix
-    path (C above 2048), with either pooling; bit-exact against the oracle's
-    selection on the GPU's own pooled values, which match the oracle's
-    pooling of the GPU's scores (max: exactly; avg: an fp32 sum of `pool`
-    terms and one division, within (pool + 1) * 2^-24 relative)."""
+    """Selection on continuous scores (C from 1 to above 2048, rows split
+    over one to four CTAs, pooling radius 0 to 511) with either pooling;
+    bit-exact against the oracle's selection on the GPU's own pooled values,
+    which match the oracle's pooling of the GPU's scores (max: exactly; avg:
+    an fp32 sum of `pool` terms and one division, within (pool + 1) * 2^-24
+    relative)."""
     import torch
     rng = np.random.default_rng(19)
     pm = P.SPK_POOL_MAX if mode == "max" else P.SPK_POOL_AVG
     for n, kk, tail, pool in [(65472, 256, 64, 7), (65472, 2048, 0, 7), (65472, 2049, 0, 7),
-                              (20000, 5000, 3, 3), (777, 1, 2, 9), (777, 776, 0, 1), (4096, 300, 0, 1023)]:
+                              (20000, 5000, 3, 3), (777, 1, 2, 9), (777, 776, 0, 1), (4096, 300, 0, 1023),
+                              (30000, 77, 0, 9)]:
         s = (rng.gamma(2.0, 1.0, size=(3, n)) * rng.random((3, 1))).astype(np.float32)
         st = torch.from_numpy(s).cuda()
         c = min(kk, n)
@@ -244,8 +245,8 @@ def test_topk_paths_on_continuous_scores(P, mode):
 
 def test_topk_refines_a_crowded_bin(P):
     """Scores in [1, 1.1) share one 12-bit key bin (sign, exponent, three
-    mantissa bits): the selection refines it by the next 12 bits before the
-    shared-memory sort; bit-exact against the oracle on the same values."""
+    mantissa bits): the selection refines it by the next 12 and then the last
+    8 bits; bit-exact against the oracle on the same values."""
     import torch
     rng = np.random.default_rng(37)
     for n, kk, tail, pool in [(65472, 256, 64, 7), (30000, 2048, 0, 1), (9999, 700, 5, 3)]:
@@ -258,6 +259,40 @@ def test_topk_refines_a_crowded_bin(P):
         for u in range(2):
             ref = oracle.topk_with_tail(oracle.maxpool(s[u].astype(np.float64), pool), kk, tail)
             assert got[u].tolist() == ref.tolist(), (n, kk, tail, pool)
+    assert P.spk_device_error() == (0, 0)
+
+
+@pytest.mark.parametrize("mode", ["max", "avg"])
+def test_topk_row_layouts(P, mode):
+    """Every way a row is laid out: one CTA (n <= 16384), clusters of 2, 4 and
+    8 CTAs (two CTAs per SM), eight CTAs of up to 40960 candidates (one per
+    SM), and the workspace kernel (longer rows, or a pooling radius beyond
+    1024); pooling radii inside and past the unrolled windows.  Integer-valued
+    scores, so ties straddle the CTA boundaries; bit-exact selection against
+    the oracle on the GPU's own pooled values."""
+    import torch
+    rng = np.random.default_rng(41)
+    pm = P.SPK_POOL_MAX if mode == "max" else P.SPK_POOL_AVG
+    for n, kk, tail, pool in [(16384, 1000, 4, 5), (16385, 1000, 0, 13), (40000, 3000, 2, 15),
+                              (100000, 5000, 3, 7), (131072, 257, 0, 1), (200000, 3000, 0, 11),
+                              (327680, 100, 1, 3), (327681, 100, 1, 3), (400000, 6000, 0, 7),
+                              (5000, 300, 1, 2049), (70000, 700, 0, 513)]:
+        s = rng.integers(0, 40, size=(2, n)).astype(np.float32) * 0.125
+        st = torch.from_numpy(s).cuda()
+        c = min(kk, n)
+        idx = torch.empty((2, c + tail), dtype=torch.int32, device="cuda")
+        pooled = torch.empty((2, n), dtype=torch.float32, device="cuda")
+        P.topk_select(st, kk, tail, idx, pool, pooled=pooled, pool_mode=pm)
+        torch.cuda.synchronize()
+        got, gp = idx.cpu().numpy(), pooled.cpu().numpy()
+        for u in range(2):
+            ref_pool = oracle.pool(s[u].astype(np.float64), pool, mode)
+            if mode == "max":
+                np.testing.assert_array_equal(gp[u], ref_pool.astype(np.float32))
+            else:
+                np.testing.assert_allclose(gp[u], ref_pool, rtol=(pool + 1) * 2.0 ** -24, atol=0)
+            own = oracle.topk_with_tail(gp[u].astype(np.float64), kk, tail)
+            assert got[u].tolist() == own.tolist(), (n, kk, tail, pool, mode)
     assert P.spk_device_error() == (0, 0)
 
 
