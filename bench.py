@@ -696,7 +696,7 @@ def run_decode(args, cfg, P, dev):
         "config": {"workload": cfg.name, "n_kv": cfg.n_kv, "units": cfg.units, "hq": hq, "head_dim": d,
                    "l2": "4 cache copies in rotation (4 x 84 MB > L2); no flush",
                    "timing": f"CUDA graph of {reps} launches replayed; events around each replay"},
-        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
+        "roofline": {"bound": "hbm", "kernel": "decode_stream_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peaks['source']} HBM copy"},
         "full_cache": None if ms_full is None else {

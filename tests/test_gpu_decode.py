@@ -2,9 +2,11 @@
 fp64 oracle: ragged row counts, both head sizes, GQA groups up to 8, the
 cache that speckv_compress leaves, and bitwise reproducibility.
 
-Tolerance: logits are bf16 products summed in fp32 and exponentiated with
-ex2.approx (relative error ~2^-22); the weighted sums run in fp32 over at most
-a few thousand rows, so the error is ~1e-6 of max|v|; the bound is 1e-4."""
+Tolerance: logits are bf16 products summed in fp32 on the tensor cores and
+exponentiated with ex2.approx (relative error ~2^-22); the weights enter the
+value product as two bf16 terms (16 significant bits: relative error
+<= 2^-17 each) and the sums run in fp32, so the error is ~1e-5 of max|v|;
+the bound is 1e-4."""
 import numpy as np
 import pytest
 
@@ -36,6 +38,8 @@ def _check(gpu, ref, vmax):
     (4, 1, 3, 14, 2, 64, 2048, 0.125),     # g = 7, head_dim 64
     (5, 1, 1, 8, 1, 64, 33, 2.0),          # g = 8 (the largest), peaked softmax
     (6, 1, 1, 3, 3, 128, 5, 0.5),          # g = 1, fewer rows than warps
+    (7, 1, 2, 16, 4, 128, 385, 0.1),       # 13 blocks: two slots per warp, uneven blocks per warp
+    (8, 1, 1, 6, 1, 64, 4097, 0.125),      # long cache at head_dim 64
 ])
 def test_decode_parity(P, case):
     import torch
