@@ -299,7 +299,7 @@ spk_status speckv_prefill_attention(const spk_speckv_shape* s, const void* q, co
   p.c0 = s->n_in - s->n_window + 1;
   p.c2 = s->scale * 1.4426950408889634f;
   p.row_tiles = static_cast<int>(tiles);
-  p.n_items = static_cast<int>(g.units * tiles);
+  p.n_items = static_cast<int>(g.units * ((tiles + 1) / 2));   // pairs of Q tiles
   p.out = out;
   p.lse2 = lse2;
   p.off_blocks = static_cast<uint8_t*>(ws);

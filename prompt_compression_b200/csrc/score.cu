@@ -63,6 +63,7 @@ constexpr int kThreads = 18 * 32;
 // pass and 2 of 8 for the column passes.
 constexpr int kPolyRowPass = 1;
 constexpr int kPolyPairsOf8 = 2;
+constexpr int kPolyPcPairsOf8 = 1;   // the SpecPC column pass (measured best)
 
 template <int MODE, int D>
 struct Cfg {
@@ -631,11 +632,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const int mc = mask_class(nb0);
                   if (mc == 0) {
                     float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-                    colsum32<kPolyPairsOf8>(v, p.c2, gs);
+                    colsum32<kPolyPcPairsOf8>(v, p.c2, gs);
                     seg_sum += fold(gs);
                   } else if (mc == 2) {
                     float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
-                    colsum32<kPolyPairsOf8, true>(v, p.c2, gs, min(32, max(0, m_lane - mod_R(p, nb0) + 1)));
+                    colsum32<kPolyPcPairsOf8, true>(v, p.c2, gs, min(32, max(0, m_lane - mod_R(p, nb0) + 1)));
                     seg_sum += fold(gs);
                   }
                 } else {

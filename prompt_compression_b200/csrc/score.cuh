@@ -85,7 +85,7 @@ struct AttnParams {
   int c0;            // head-local row i sees keys [0, c0 + i) of input + lookahead
   float c2;          // scale * log2(e)
   int row_tiles;     // 128-row Q tiles per unit
-  int n_items;       // units * row_tiles
+  int n_items;       // units * ceil(row_tiles / 2): an item is a pair of Q tiles
   void* out;         // bf16 [units][rows][head_dim]
   float* lse2;       // fp32 [units][rows] or null: log2-domain LSE over the input keys
   uint8_t* off_blocks;   // row offsets for the column pass (row_tiles blocks per unit) or null

@@ -103,6 +103,7 @@ def _check(P, qb, kb, vb, nw, scale=1.0):
     (5, 1, 1, 2, 1, 64, 129, 0, 200),       # no window; two lookahead tiles (the second ragged)
     (6, 1, 1, 4, 4, 128, 96, 96, 4),        # window covers the whole input
     (7, 1, 1, 16, 1, 128, 1500, 64, 64),    # g * R = 2048 rows
+    (10, 1, 1, 6, 2, 128, 800, 60, 60),     # 360 rows: three Q tiles, the second pair's B tile empty
 ])
 def test_prefill_attention_parity(P, case):
     seed, B, L, hq, hkv, d, n_in, nw, nl = case
