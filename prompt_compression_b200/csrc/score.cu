@@ -581,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // (Only m_lane stays live through the loop; the warp-wide facts are
           // recomputed per group, which costs a vote in the common case.)
           const int m_lane = masked_key ? j - p.c0 : -1;
+          const bool warp_masked = __any_sync(0xffffffffu, m_lane >= 0);   // some key of the warp is masked
           // 0: no row masked, 1: every row masked, 2: leading rows masked,
           // 3: the group wraps into the next head (per-row test)
           auto mask_class = [&](int nb0) -> int {
@@ -661,6 +662,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 32 columns per TMEM wait keeps the live registers within budget
             const uint32_t taddr = tbase + acc_buf * 128 + col0;
             if (width == 0) release_acc();
+            if (MODE == MODE_COLSUM_PC && width > 0 && !warp_masked) {
+              // SpecPC, no key of the warp masked for any row: when the
+              // warp's columns are real rows of one query head, one head
+              // switch and one fold for all of them
+              const int nb0 = bt * 128 + col0;
+              const int h0 = div_R(p, nb0);
+              if (nb0 + width <= p.rows && h0 == div_R(p, nb0 + width - 1)) {
+                if (h0 != cur_head) {
+                  if (cur_head >= 0) my_acc[(head0 + cur_head) * 256 + r] += seg_sum;
+                  cur_head = h0;
+                  seg_sum = 0.f;
+                }
+                float2 gs[4] = {f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+                for (int g = 0; g < width; g += 32) {
+                  uint32_t v[32];
+                  __syncwarp();
+                  tmem_ld32(taddr + g, v);
+                  tmem_ld_wait(v);
+                  if (g + 32 >= width) release_acc();
+                  colsum32<kPolyPcPairsOf8>(v, p.c2, gs);
+                }
+                seg_sum += fold(gs);
+                next_acc();
+                continue;
+              }
+            }
             for (int g = 0; g < width; g += 32) {
               uint32_t v[32];
               __syncwarp();
