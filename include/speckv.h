@@ -191,7 +191,7 @@ spk_status speckv_prefill_attention(const spk_speckv_shape* shape, const void* q
  * A vertical or slash entry outside [0, n) is ignored and recorded as
  * SPK_ERR_ARG in the device error word; unsorted lists give wrong results.
  * Probabilities enter the P.V product as bf16 (fp32 accumulation).
- * Supported: head_dim in {64, 128}; hq % hkv == 0; 1 <= n_q <= n <= 131072;
+ * Supported: head_dim in {64, 128}; hq % hkv == 0; 1 <= n_q <= n <= 65536;
  * n_vertical <= 4096; n_slash <= n.
  * ------------------------------------------------------------------------ */
 typedef struct {

@@ -381,7 +381,7 @@ spk_status vs_sparse_attention(const spk_vs_shape* s, const void* q, const void*
   p.n_s = s->n_slash;
   p.c2 = s->scale * 1.4426950408889634f;
   p.row_blocks = (s->n_q + 127) / 128;
-  p.n_items = static_cast<int>(units * g * p.row_blocks);
+  p.n_items = static_cast<int>(units * ((g + 1) / 2) * p.row_blocks);   // pairs of query heads
   p.vert = vertical;
   p.slash = slash;
   p.out = out;

@@ -95,7 +95,7 @@ cudaError_t launch_attn(int head_dim, const CUtensorMap (&maps)[5], const AttnPa
                         cudaStream_t stream);
 
 // Vertical-Slash sparse prefill attention (vs.cu)
-constexpr int kVsMaxN = 131072;     // keys per unit (the pattern's bitmaps live in shared memory)
+constexpr int kVsMaxN = 65536;      // keys per unit (the pattern's bitmaps live in shared memory)
 constexpr int kVsMaxVert = 4096;    // vertical columns per unit
 struct VsParams {
   int n;             // keys per unit
@@ -104,7 +104,7 @@ struct VsParams {
   int n_v, n_s;      // vertical columns and slash offsets per unit
   float c2;          // scale * log2(e)
   int row_blocks;    // ceil(n_q / 128)
-  int n_items;       // units * g * row_blocks
+  int n_items;       // units * ceil(g / 2) * row_blocks: an item is a pair of query heads
   const int* vert;   // [units][n_v] ascending key indices
   const int* slash;  // [units][n_s] ascending offsets
   void* out;         // bf16 [units * g][n_q][d]

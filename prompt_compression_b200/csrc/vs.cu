@@ -12,8 +12,12 @@
 // Query rows are the last n_q positions of the n-token sequence, every query
 // head of the unit's GQA group.
 //
-// Work decomposition: an item is one query head's 128-row tile (positions
-// p0 .. p0 + 127).  Its keys come in 128-key tiles of two kinds:
+// Work decomposition: an item is a pair of query heads of one unit's GQA
+// group (heads 2 hp and 2 hp + 1) over one 128-row block (positions
+// p0 .. p0 + 127).  The two heads have the same rows, hence the same key
+// tiles and the same masks: they share every K/V tile, and two softmax
+// warpgroups (one per head) work in ping-pong, each while the other head's
+// products run.  The item's keys come in 128-key tiles of two kinds:
 //   slash tiles    -- tiles of K/V that a slash diagonal (or the self
 //                     diagonal) crosses for some row of the item: tile t is
 //                     crossed iff some o in S u {0} lies in
@@ -26,10 +30,12 @@
 // word per 32 keys, the slash word bit-reversed); in a vertical tile a key is
 // visible iff j <= p and its K/V tile was not a slash tile of the item (there
 // it was already counted).  The pipeline is the prefill attention's: a TMA
-// producer warp, a single-thread UMMA issuer (S = Q K^T from shared memory,
-// O += P V with P in TMEM as bf16 and V MN-major from shared memory) and
-// four softmax warps (thread = row; lazy rescale of O when the running max
-// moves by more than 2^8).  Every role derives the same tile sequence.
+// producer warp (both heads' Q tiles, then the K/V tiles), a single-thread
+// UMMA issuer (per tile: O_A += P_A V, S_A(next), O_B += P_B V, S_B(next);
+// S = Q K^T from shared memory, O += P V with P in TMEM as bf16 and V
+// MN-major from shared memory) and eight softmax warps (thread = row; S read
+// in 64-column halves; lazy rescale of O when the running max moves by more
+// than 2^8).  Every role derives the same tile sequence.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -39,10 +45,10 @@
 namespace spk {
 namespace {
 
-constexpr int kVsSoftmaxWarps = 4;
-constexpr int kVsProducerWarp = 4;
-constexpr int kVsMmaWarp = 5;
-constexpr int kVsThreads = 6 * 32;
+constexpr int kVsGroupWarps = 4;       // softmax warps per head of the pair (two groups)
+constexpr int kVsProducerWarp = 8;
+constexpr int kVsMmaWarp = 9;
+constexpr int kVsThreads = 10 * 32;
 constexpr float kVsRescale = 8.f;
 constexpr int kVsPolyOf8 = 2;          // exponential pairs (of 8) evaluated on the FMA pipe
 
@@ -52,7 +58,8 @@ struct VsCfg {
   static constexpr int kAtoms = D / 64;
   static constexpr int kStages = 2;
   static constexpr int kBitWords = kVsMaxN / 32;
-  static constexpr int kSmemBytes = 1024 + kTileBytes + 2 * kStages * kTileBytes + 2 * kBitWords * 4 + kVsMaxVert * 4;
+  static constexpr int kSmemBytes =
+      1024 + 2 * kTileBytes + 2 * kStages * kTileBytes + 2 * kBitWords * 4 + kVsMaxVert * 4;   // Q x 2, K and V rings
   static_assert(kSmemBytes <= 227 * 1024 - 2048, "fits one CTA");
 };
 
@@ -75,6 +82,16 @@ __device__ __forceinline__ void vs_tmem_st32(uint32_t taddr, const uint32_t (&r)
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane from registers.
+__device__ __forceinline__ void vs_tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 
@@ -146,15 +163,16 @@ __global__ void __launch_bounds__(kVsThreads, 1)
   using C = VsCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* const Q_s = smem;
-  uint8_t* const K_s = smem + C::kTileBytes;
+  uint8_t* const Q_s = smem;                                    // [2 heads]
+  uint8_t* const K_s = smem + 2 * C::kTileBytes;
   uint8_t* const V_s = K_s + C::kStages * C::kTileBytes;
   uint32_t* const vbits = reinterpret_cast<uint32_t*>(V_s + C::kStages * C::kTileBytes);   // V as a bitmap
   uint32_t* const sbits = vbits + C::kBitWords;                                           // S as a bitmap
   int* const vidx_s = reinterpret_cast<int*>(sbits + C::kBitWords);                      // V, ascending
 
+  // per Q tile x (0: A, 1: B): s_full[x], p_full[x] (4 warps), pv_done[x], o_empty[x] (4 warps)
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
-      p_full[2], pv_done, o_empty, done_bar, soft_bar;
+      p_full[2], pv_done[2], o_empty[2], done_bar, soft_bar;
   __shared__ uint32_t slash_tiles[kVsMaxN / 128 / 32];   // tiles of the current item that were slash tiles
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
@@ -163,6 +181,7 @@ __global__ void __launch_bounds__(kVsThreads, 1)
   const int lane = threadIdx.x & 31;
   const int n = p.n;
   const int n_words = (n + 31) >> 5;
+  const int hpairs = (p.g + 1) / 2;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
@@ -170,12 +189,11 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
-      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kVsSoftmaxWarps);
+      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kVsGroupWarps);
+      mbar_init(&pv_done[s], 1); mbar_init(&o_empty[s], kVsGroupWarps);
     }
-    mbar_init(&pv_done, 1);
-    mbar_init(&o_empty, kVsSoftmaxWarps);
     mbar_init(&done_bar, 1);
-    mbar_init(&soft_bar, kVsSoftmaxWarps);
+    mbar_init(&soft_bar, 2 * kVsGroupWarps);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -198,12 +216,14 @@ __global__ void __launch_bounds__(kVsThreads, 1)
   const uint32_t tmem_base = tmem_holder;
   volatile int* abort_v = &abort_flag;
 
-  // item -> (unit, query head of the group, row block); rows' positions p0 .. p_last
-  auto item_geom = [&](int item, int& u, int& qh, int& rb, int& p0, int& p_last) {
+  // item -> (unit, head pair, row block); rows' positions p0 .. p_last; the
+  // pair's query heads 2 hp and 2 hp + 1 of the group share every key tile
+  // and every mask
+  auto item_geom = [&](int item, int& u, int& hp, int& rb, int& p0, int& p_last) {
     rb = item % p.row_blocks;
-    const int hu = item / p.row_blocks;   // u * g + head
-    u = hu / p.g;
-    qh = hu;
+    const int hu = item / p.row_blocks;   // u * hpairs + hp
+    u = hu / hpairs;
+    hp = hu % hpairs;
     p0 = n - p.n_q + rb * 128;
     p_last = n - p.n_q + min(rb * 128 + 127, p.n_q - 1);
   };
@@ -217,7 +237,9 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     return n_slash + (cv + 127) / 128;
   };
 
-  if (warp == kVsProducerWarp) {
+  if (warp > kVsMmaWarp) {
+    // (no other warps)
+  } else if (warp == kVsProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
@@ -225,13 +247,18 @@ __global__ void __launch_bounds__(kVsThreads, 1)
       int items_done = 0;
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1}, q_last = -1;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
-        int u, qh, rb, p0, p_last;
-        item_geom(item, u, qh, rb, p0, p_last);
+        int u, hp, rb, p0, p_last;
+        item_geom(item, u, hp, rb, p0, p_last);
         int n_slash, cv;
         const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
         if (!(ok = mbar_wait(&q_empty, (items_done & 1) ^ 1, abort_v, vs_site(0, 0)))) break;
-        mbar_arrive_expect_tx(&q_full, C::kTileBytes);
-        for (int a = 0; a < C::kAtoms; ++a) tma_load_3d(Q_s + a * 16384, &qmap, &q_full, a * 64, rb * 128, qh);
+        mbar_arrive_expect_tx(&q_full, 2 * C::kTileBytes);
+        for (int x = 0; x < 2; ++x) {
+          // a missing second head (odd g) loads the next head's rows (or zeros): never stored
+          const int qh = u * p.g + 2 * hp + x;
+          for (int a = 0; a < C::kAtoms; ++a)
+            tma_load_3d(Q_s + x * C::kTileBytes + a * 16384, &qmap, &q_full, a * 64, rb * 128, qh);
+        }
         q_last = items_done & 1;
         const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
         int t = p_last >> 7, sa = 0;
@@ -263,59 +290,64 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     }
   } else if (warp == kVsMmaWarp) {
     // ------------------------------------------------------------ UMMA issuer
+    // Order per key tile t: O_A += P_A V(t), S_A(t+1), O_B += P_B V(t), S_B(t+1)
+    // (each softmax group works while the other's products run; S_x(t+1)
+    // follows O_x's product of tile t, so O_x is quiescent once it lands).
     if (lane == 0) {
       bool ok = true;
       uint32_t T = 0;
       int items_done = 0;
       const uint32_t idesc_s = idesc_bf16_f32(128, 128);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 64) | (1u << 16);   // B (V) MN-major
-      const uint64_t q_desc = sw128_kmajor_desc(smem_u32(Q_s));
-      auto issue_s = [&](uint32_t Ti) -> bool {
+      auto issue_s = [&](int x, uint32_t Ti) -> bool {
         const int st = Ti & 1;
-        if (!mbar_wait(&k_full[st], (Ti >> 1) & 1, abort_v, vs_site(1, 1))) return false;
+        if (x == 0 && !mbar_wait(&k_full[st], (Ti >> 1) & 1, abort_v, vs_site(1, 1))) return false;
         tc_fence_after();
+        const uint64_t q_desc = sw128_kmajor_desc(smem_u32(Q_s + x * C::kTileBytes));
         const uint64_t k_desc = sw128_kmajor_desc(smem_u32(K_s + st * C::kTileBytes));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-          umma_bf16_ss(tmem_base + st * 128, q_desc + koff, k_desc + koff, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem_base + x * 256, q_desc + koff, k_desc + koff, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[st]);
-        umma_commit(&k_empty[st]);
+        umma_commit(&s_full[x]);
+        if (x == 1) umma_commit(&k_empty[st]);
+        return true;
+      };
+      auto issue_pv = [&](int x, uint32_t Ti, int t) -> bool {
+        const int st = Ti & 1;
+        if (!mbar_wait(&p_full[x], Ti & 1, abort_v, vs_site(1, 4 + x))) return false;
+        if (x == 0 && !mbar_wait(&v_full[st], (Ti >> 1) & 1, abort_v, vs_site(1, 6))) return false;
+        if (t == 0 && items_done > 0 && !mbar_wait(&o_empty[x], (items_done - 1) & 1, abort_v, vs_site(1, 7 + x)))
+          return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(V_s + st * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+          for (int a = 0; a < C::kAtoms; ++a) {
+            const uint64_t v_desc = vs_mnmajor_desc(v_base + a * 16384 + kk * 2048, 16384);
+            umma_bf16_ts(tmem_base + x * 256 + 128 + a * 64, tmem_base + x * 256 + 64 + kk * 8, v_desc, idesc_pv,
+                         (t > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&pv_done[x]);
+        if (x == 1) umma_commit(&v_empty[st]);
         return true;
       };
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
-        int u, qh, rb, p0, p_last;
-        item_geom(item, u, qh, rb, p0, p_last);
+        int u, hp, rb, p0, p_last;
+        item_geom(item, u, hp, rb, p0, p_last);
         int n_slash, cv;
         const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
         if (!(ok = mbar_wait(&q_full, items_done & 1, abort_v, vs_site(1, 0)))) break;
-        if (T >= 1 && !(ok = mbar_wait(&pv_done, (T - 1) & 1, abort_v, vs_site(1, 2)))) break;
-        if (!(ok = issue_s(T))) break;
+        if (!(ok = issue_s(0, T)) || !(ok = issue_s(1, T))) break;
         for (int t = 0; ok && t < n_tiles; ++t) {
           const uint32_t Tc = T + t;
-          if (t + 1 < n_tiles) {
-            if (Tc >= 1 && !(ok = mbar_wait(&pv_done, (Tc - 1) & 1, abort_v, vs_site(1, 3)))) break;
-            if (!(ok = issue_s(Tc + 1))) break;
-          }
-          const int st = Tc & 1;
-          if (!(ok = mbar_wait(&p_full[st], (Tc >> 1) & 1, abort_v, vs_site(1, 4)))) break;
-          if (!(ok = mbar_wait(&v_full[st], (Tc >> 1) & 1, abort_v, vs_site(1, 5)))) break;
-          if (t == 0 && items_done > 0 && !(ok = mbar_wait(&o_empty, (items_done - 1) & 1, abort_v, vs_site(1, 6))))
-            break;
-          tc_fence_after();
-          const uint32_t v_base = smem_u32(V_s + st * C::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-            for (int a = 0; a < C::kAtoms; ++a) {
-              const uint64_t v_desc = vs_mnmajor_desc(v_base + a * 16384 + kk * 2048, 16384);
-              umma_bf16_ts(tmem_base + 256 + a * 64, tmem_base + st * 128 + kk * 8, v_desc, idesc_pv,
-                           (t > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
-          umma_commit(&v_empty[st]);
-          umma_commit(&pv_done);
+          if (!(ok = issue_pv(0, Tc, t))) break;
+          if (t + 1 < n_tiles && !(ok = issue_s(0, Tc + 1))) break;
+          if (!(ok = issue_pv(1, Tc, t))) break;
+          if (t + 1 < n_tiles && !(ok = issue_s(1, Tc + 1))) break;
         }
         if (!ok) break;
         umma_commit(&q_empty);
@@ -326,18 +358,20 @@ __global__ void __launch_bounds__(kVsThreads, 1)
       mbar_wait(&done_bar, 0, &never, vs_site(1, 9), 100000000ull);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int tid = threadIdx.x;                        // 0 .. 127
-    const int r = warp * 32 + lane;                     // row within the Q tile = TMEM lane
-    const uint32_t tlane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    // ------------------------------------------------------------ softmax groups
+    const int x = warp >> 2;                            // head of the pair (Q tile)
+    const int wq = warp & 3;
+    const int tid = threadIdx.x;                        // 0 .. 255 over both groups
+    const int r = wq * 32 + lane;                       // row within the Q tile = TMEM lane
+    const uint32_t tlane = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + x * 256;   // S; O at +128
     bool ok = true;
     uint32_t T = 0;
     int items_done = 0, loaded_unit = -1;
     auto wait_all = [&](uint64_t* bar, uint32_t parity, int which) -> bool {
-      bool w = mbar_wait(bar, parity, abort_v, vs_site(2, which));
+      bool w = mbar_wait(bar, parity, abort_v, vs_site(2 + x, which));
       return __all_sync(0xffffffffu, w);
     };
-    // the four softmax warps meet (their shared-memory writes before it are
+    // the eight softmax warps meet (their shared-memory writes before it are
     // visible after it); a bounded wait, so an aborted CTA cannot strand a warp
     uint32_t soft_phase = 0;
     auto softmax_sync = [&]() -> bool {
@@ -348,42 +382,43 @@ __global__ void __launch_bounds__(kVsThreads, 1)
       return w;
     };
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
-      int u, qh, rb, p0, p_last;
-      item_geom(item, u, qh, rb, p0, p_last);
+      int u, hp, rb, p0, p_last;
+      item_geom(item, u, hp, rb, p0, p_last);
       int n_slash, cv;
       const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
       // this unit's pattern as bitmaps (and V as a list), and no slash tile yet
       if (!(ok = softmax_sync())) break;                // the previous item is done with them
       if (u != loaded_unit) {
-        for (int w = tid; w < n_words; w += 128) { vbits[w] = 0u; sbits[w] = 0u; }
+        for (int w = tid; w < n_words; w += 256) { vbits[w] = 0u; sbits[w] = 0u; }
         if (!(ok = softmax_sync())) break;
         const int* vg = p.vert + static_cast<size_t>(u) * p.n_v;
         const int* sg = p.slash + static_cast<size_t>(u) * p.n_s;
-        for (int x = tid; x < p.n_v; x += 128) {
-          const int j = __ldg(vg + x);
-          vidx_s[x] = j;
+        for (int i = tid; i < p.n_v; i += 256) {
+          const int j = __ldg(vg + i);
+          vidx_s[i] = j;
           if (j >= 0 && j < n) atomicOr(&vbits[j >> 5], 1u << (j & 31));
           else record_error(SPK_DEVERR_INDEX, u);
         }
-        for (int x = tid; x < p.n_s; x += 128) {
-          const int o = __ldg(sg + x);
+        for (int i = tid; i < p.n_s; i += 256) {
+          const int o = __ldg(sg + i);
           if (o >= 0 && o < n) atomicOr(&sbits[o >> 5], 1u << (o & 31));
           else record_error(SPK_DEVERR_INDEX, u);
         }
         loaded_unit = u;
       }
-      for (int w = tid; w < kVsMaxN / 128 / 32; w += 128) slash_tiles[w] = 0u;
+      for (int w = tid; w < kVsMaxN / 128 / 32; w += 256) slash_tiles[w] = 0u;
       if (!(ok = softmax_sync())) break;
 
+      const int h = 2 * hp + x;                         // head of the group
+      const int qh = u * p.g + h;
       const int i_row = rb * 128 + r;
-      const bool live = i_row < p.n_q;
-      const int pos = live ? n - p.n_q + i_row : n - 1;
+      const bool live = i_row < p.n_q && h < p.g;
+      const int pos = i_row < p.n_q ? n - p.n_q + i_row : n - 1;
       const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
       int wt = p_last >> 7, wa = 0;                     // this role's walk over the slash tiles
       float m = -INFINITY, l = 0.f;
       for (int t = 0; ok && t < n_tiles; ++t) {
         const uint32_t Tc = T + t;
-        const int buf = Tc & 1;
         const bool slash = t < n_slash;
         int j0 = 0;
         if (slash) {
@@ -412,10 +447,10 @@ __global__ void __launch_bounds__(kVsThreads, 1)
           const int vis_n = upper_bound_le(vidx_s + base, cnt, pos);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const int x = 32 * c + lane;
+            const int xx = 32 * c + lane;
             bool okc = false;
-            if (x < cnt) {
-              const int j = vidx_s[base + x];
+            if (xx < cnt) {
+              const int j = vidx_s[base + xx];
               okc = j >= 0 && j < n && !((slash_tiles[j >> 12] >> ((j >> 7) & 31)) & 1u);
             }
             const uint32_t dedupe = __ballot_sync(0xffffffffu, okc);
@@ -424,46 +459,50 @@ __global__ void __launch_bounds__(kVsThreads, 1)
             vis[c] = dedupe & pre;
           }
         }
-        if (!(ok = wait_all(&s_full[buf], (Tc >> 1) & 1, 0))) break;
+        if (!(ok = wait_all(&s_full[x], Tc & 1, 0))) break;
         tc_fence_after();
-        float s[128];
-        {
-          uint32_t a0[32], a1[32];
-          tmem_ld32(tlane + buf * 128, a0);
-          tmem_ld32(tlane + buf * 128 + 32, a1);
-          tmem_ld_wait2(a0, a1);
+        // S columns [0, 64) then [64, 128), masked: the row max
+        auto mask64 = [&](uint32_t (&a0)[32], uint32_t (&a1)[32], uint32_t v0, uint32_t v1) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            s[k] = ((vis[0] >> k) & 1u) ? __uint_as_float(a0[k]) : -INFINITY;
-            s[32 + k] = ((vis[1] >> k) & 1u) ? __uint_as_float(a1[k]) : -INFINITY;
+            if (!((v0 >> k) & 1u)) a0[k] = __float_as_uint(-INFINITY);
+            if (!((v1 >> k) & 1u)) a1[k] = __float_as_uint(-INFINITY);
           }
-          tmem_ld32(tlane + buf * 128 + 64, a0);
-          tmem_ld32(tlane + buf * 128 + 96, a1);
-          tmem_ld_wait2(a0, a1);
+        };
+        auto max64 = [&](const uint32_t (&a0)[32], const uint32_t (&a1)[32], float mx) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            s[64 + k] = ((vis[2] >> k) & 1u) ? __uint_as_float(a0[k]) : -INFINITY;
-            s[96 + k] = ((vis[3] >> k) & 1u) ? __uint_as_float(a1[k]) : -INFINITY;
+          for (int k = 0; k < 32; k += 4) {
+            mx = fmaxf(mx, max3f(__uint_as_float(a0[k]), __uint_as_float(a0[k + 1]),
+                                 fmaxf(__uint_as_float(a0[k + 2]), __uint_as_float(a0[k + 3]))));
+            mx = fmaxf(mx, max3f(__uint_as_float(a1[k]), __uint_as_float(a1[k + 1]),
+                                 fmaxf(__uint_as_float(a1[k + 2]), __uint_as_float(a1[k + 3]))));
           }
-        }
+          return mx;
+        };
         float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 128; k += 4) mx = fmaxf(mx, max3f(s[k], s[k + 1], fmaxf(s[k + 2], s[k + 3])));
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t a0[32], a1[32];
+          tmem_ld32(tlane + 64 * hh, a0);
+          tmem_ld32(tlane + 64 * hh + 32, a1);
+          tmem_ld_wait2(a0, a1);
+          mask64(a0, a1, vis[2 * hh], vis[2 * hh + 1]);
+          mx = max64(a0, a1, mx);
+        }
         const float mt = mx * p.c2;
         const bool need = mx != -INFINITY && mt > m + kVsRescale;
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = need ? ex2_approx(m - mt) : 1.f;
           if (t > 0) {
-            if (!(ok = wait_all(&pv_done, (Tc - 1) & 1, 1))) break;
-            tc_fence_after();
+            // O holds the P.V products of tiles 0 .. t-1, all retired (S(t) was issued after them)
 #pragma unroll 1
             for (int ch = 0; ch < D / 32; ++ch) {
               uint32_t o[32];
-              tmem_ld32(tlane + 256 + ch * 32, o);
+              tmem_ld32(tlane + 128 + ch * 32, o);
               tmem_ld_wait(o);
 #pragma unroll
               for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-              vs_tmem_st32(tlane + 256 + ch * 32, o);
+              vs_tmem_st32(tlane + 128 + ch * 32, o);
             }
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           }
@@ -472,46 +511,58 @@ __global__ void __launch_bounds__(kVsThreads, 1)
             m = mt;
           }
         }
-        // P = 2^(c2 s - m): masked keys (s = -inf) give 0; a row that has
-        // seen no key yet (m = -inf) has only masked keys here
-        // (the FMA-pipe exponential turns a masked key into 2^-126 instead of
-        // 0: far below the rounding of the sum and of O, and wiped by the
-        // rescale when a row sees its first key)
+        // P = 2^(c2 s - m) into TMEM columns [64, 128) of the S buffer: S
+        // columns [64, 128) are read again and theirs go to [96, 128), then
+        // those of S columns [0, 64) to [64, 96) -- every column written has
+        // been read.  Masked keys (s = -inf) give 0; a row
+        // that has seen no key yet (m = -inf) has only masked keys here (the
+        // FMA-pipe exponential turns a masked key into 2^-126 instead of 0:
+        // far below the rounding of the sum and of O, and wiped by the
+        // rescale when the row sees its first key).
         const float mm = m == -INFINITY ? 0.f : m;
         const float2 c2v = f2(p.c2, p.c2), nm = f2(-mm, -mm);
         float2 acc2 = f2(0.f, 0.f);
-        uint32_t pk[64];
+        // 32 S values -> 16 packed P words at TMEM column `col`
+        auto exp32 = [&](const uint32_t (&a)[32], uint32_t col) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          const float2 tt = __ffma2_rn(f2(s[2 * k], s[2 * k + 1]), c2v, nm);
-          const float2 e = ((k & 7) < kVsPolyOf8) ? exp2_fma_pair(tt) : exp2_mufu_pair(tt);
-          acc2 = __fadd2_rn(acc2, e);
-          pk[k] = vs_pack_bf16(e.x, e.y);
+          for (int k = 0; k < 16; ++k) {
+            const float2 tt = __ffma2_rn(f2(__uint_as_float(a[2 * k]), __uint_as_float(a[2 * k + 1])), c2v, nm);
+            const float2 e = ((k & 7) < kVsPolyOf8) ? exp2_fma_pair(tt) : exp2_mufu_pair(tt);
+            acc2 = __fadd2_rn(acc2, e);
+            pk[k] = vs_pack_bf16(e.x, e.y);
+          }
+          vs_tmem_st16(col, pk);
+        };
+#pragma unroll 1
+        for (int hh = 1; hh >= 0; --hh) {
+          uint32_t a0[32], a1[32];
+          tmem_ld32(tlane + 64 * hh, a0);
+          tmem_ld32(tlane + 64 * hh + 32, a1);
+          tmem_ld_wait2(a0, a1);
+          mask64(a0, a1, vis[2 * hh], vis[2 * hh + 1]);
+          exp32(a0, tlane + 64 + 32 * hh);
+          exp32(a1, tlane + 64 + 32 * hh + 16);
         }
         l += acc2.x + acc2.y;
-        {
-          uint32_t (&p0r)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-          uint32_t (&p1r)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-          vs_tmem_st32(tlane + buf * 128, p0r);
-          vs_tmem_st32(tlane + buf * 128 + 32, p1r);
-        }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[buf]);
+        if (lane == 0) mbar_arrive(&p_full[x]);
       }
       if (!ok) break;
+      // S(Tl) landed after P.V(Tl - 1) retired: the P.V barrier's phase for
+      // P.V(Tl) is the newest or the one just completed
       const uint32_t Tl = T + n_tiles - 1;
-      if (Tl >= 1 && !(ok = wait_all(&pv_done, (Tl - 1) & 1, 2))) break;
-      if (!(ok = wait_all(&pv_done, Tl & 1, 3))) break;
+      if (!(ok = wait_all(&pv_done[x], Tl & 1, 3))) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                            (static_cast<size_t>(qh) * p.n_q + (live ? i_row : 0)) * D;
+                            (static_cast<size_t>(live ? qh : 0) * p.n_q + (live ? i_row : 0)) * D;
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
-        tmem_ld32(tlane + 256 + ch * 32, o);
+        tmem_ld32(tlane + 128 + ch * 32, o);
         tmem_ld_wait(o);
         if (live) {
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
@@ -528,7 +579,7 @@ __global__ void __launch_bounds__(kVsThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty);
+      if (lane == 0) mbar_arrive(&o_empty[x]);
       if (p.lse2 != nullptr && live) p.lse2[static_cast<size_t>(qh) * p.n_q + i_row] = m + lg2_approx(l);
       T += n_tiles;
     }
