@@ -121,16 +121,6 @@ __device__ __forceinline__ int next_slash_tile(const int* __restrict__ S, int n_
 }
 
 // Number of entries of the ascending array x[0, n) that are <= v.
-__device__ __forceinline__ int upper_bound_le(const int* x, int n, int v) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (x[mid] <= v) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
-}
-
 __device__ __forceinline__ int upper_bound_le_global(const int* __restrict__ x, int n, int v) {
   int lo = 0, hi = n;
   while (lo < hi) {
@@ -443,19 +433,28 @@ __global__ void __launch_bounds__(kVsThreads, 1)
           const int base = 128 * (t - n_slash);         // gathered rows of this vertical tile
           const int cnt = min(128, cv - base);
           __syncwarp();
-          // keys of slash tiles were counted there; vertical keys <= pos only
-          const int vis_n = upper_bound_le(vidx_s + base, cnt, pos);
+          // keys of slash tiles were counted there; vertical keys <= pos
+          // only.  The warp's rows are the consecutive positions pos0 + lane
+          // (rows past n_q are never stored), and the tile's keys ascend, so
+          // the keys <= pos of a 32-key chunk are a prefix of it, of length
+          // (keys < pos0) + (keys in [pos0, pos0 + lane]).
+          const int pos0 = __shfl_sync(0xffffffffu, pos, 0);
+          const uint32_t upto = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const int xx = 32 * c + lane;
             bool okc = false;
+            int dj = 1 << 30;                           // key - pos0 (past the tile: never visible)
             if (xx < cnt) {
               const int j = vidx_s[base + xx];
               okc = j >= 0 && j < n && !((slash_tiles[j >> 12] >> ((j >> 7) & 31)) & 1u);
+              dj = j - pos0;
             }
             const uint32_t dedupe = __ballot_sync(0xffffffffu, okc);
-            const int lim = vis_n - 32 * c;
-            const uint32_t pre = lim <= 0 ? 0u : (lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u));
+            const int below = __popc(__ballot_sync(0xffffffffu, dj < 0));
+            const uint32_t near = __reduce_or_sync(0xffffffffu, (dj >= 0 && dj < 32) ? (1u << dj) : 0u);
+            const int k = below + __popc(near & upto);   // keys of the chunk <= pos0 + lane
+            const uint32_t pre = k >= 32 ? 0xffffffffu : ((1u << k) - 1u);
             vis[c] = dedupe & pre;
           }
         }
@@ -486,7 +485,7 @@ __global__ void __launch_bounds__(kVsThreads, 1)
           tmem_ld32(tlane + 64 * hh, a0);
           tmem_ld32(tlane + 64 * hh + 32, a1);
           tmem_ld_wait2(a0, a1);
-          mask64(a0, a1, vis[2 * hh], vis[2 * hh + 1]);
+          mask64(a0, a1, hh ? vis[2] : vis[0], hh ? vis[3] : vis[1]);
           mx = max64(a0, a1, mx);
         }
         const float mt = mx * p.c2;
@@ -540,7 +539,7 @@ __global__ void __launch_bounds__(kVsThreads, 1)
           tmem_ld32(tlane + 64 * hh, a0);
           tmem_ld32(tlane + 64 * hh + 32, a1);
           tmem_ld_wait2(a0, a1);
-          mask64(a0, a1, vis[2 * hh], vis[2 * hh + 1]);
+          mask64(a0, a1, hh ? vis[2] : vis[0], hh ? vis[3] : vis[1]);
           exp32(a0, tlane + 64 + 32 * hh);
           exp32(a1, tlane + 64 + 32 * hh + 16);
         }
