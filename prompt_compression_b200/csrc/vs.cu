@@ -461,11 +461,18 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         if (!(ok = wait_all(&s_full[x], Tc & 1, 0))) break;
         tc_fence_after();
         // S columns [0, 64) then [64, 128), masked: the row max
+        // (a word every lane sees whole -- the common case in vertical
+        // tiles -- needs no select)
         auto mask64 = [&](uint32_t (&a0)[32], uint32_t (&a1)[32], uint32_t v0, uint32_t v1) {
+          if (__any_sync(0xffffffffu, v0 != 0xffffffffu)) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (!((v0 >> k) & 1u)) a0[k] = __float_as_uint(-INFINITY);
-            if (!((v1 >> k) & 1u)) a1[k] = __float_as_uint(-INFINITY);
+            for (int k = 0; k < 32; ++k)
+              if (!((v0 >> k) & 1u)) a0[k] = __float_as_uint(-INFINITY);
+          }
+          if (__any_sync(0xffffffffu, v1 != 0xffffffffu)) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (!((v1 >> k) & 1u)) a1[k] = __float_as_uint(-INFINITY);
           }
         };
         auto max64 = [&](const uint32_t (&a0)[32], const uint32_t (&a1)[32], float mx) {

@@ -296,6 +296,26 @@ def test_topk_row_layouts(P, mode):
     assert P.spk_device_error() == (0, 0)
 
 
+def test_topk_degenerate_counts_on_clusters(P):
+    """C = 0 (the window only, with the pooled output requested) and C >= n
+    (every candidate) on rows split over clusters of 2, 4 and 8 CTAs."""
+    import torch
+    rng = np.random.default_rng(43)
+    for n, kk, tail, pool in [(40000, 0, 5, 7), (100000, 0, 0, 3), (50000, 50000, 3, 5), (200000, 250000, 2, 7)]:
+        s = rng.random((2, n)).astype(np.float32)
+        st = torch.from_numpy(s).cuda()
+        c = min(kk, n)
+        idx = torch.empty((2, c + tail), dtype=torch.int32, device="cuda")
+        pooled = torch.empty((2, n), dtype=torch.float32, device="cuda")
+        P.topk_select(st, kk, tail, idx, pool, pooled=pooled)
+        torch.cuda.synchronize()
+        got, gp = idx.cpu().numpy(), pooled.cpu().numpy()
+        for u in range(2):
+            np.testing.assert_array_equal(gp[u], oracle.maxpool(s[u].astype(np.float64), pool).astype(np.float32))
+            assert got[u].tolist() == list(range(c)) + list(range(n, n + tail)), (n, kk, tail)
+    assert P.spk_device_error() == (0, 0)
+
+
 def test_speckv_avg_pool_end_to_end(P):
     """speckv_compress with average pooling: scores against the oracle, the
     selection bit-exact on the GPU's own pooled values and tie-tolerant
