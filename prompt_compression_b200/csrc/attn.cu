@@ -54,7 +54,7 @@ constexpr int kAttnProducerWarp = 8;
 constexpr int kAttnMmaWarp = 9;
 constexpr int kAttnThreads = 10 * 32;
 constexpr float kRescaleLog2 = 8.f;    // lazy rescale threshold (P <= 2^8)
-constexpr int kAttnPolyOf8 = 2;        // exponential pairs (of 8) evaluated on the FMA pipe
+constexpr int kAttnPolyOf8 = 1;        // exponential pairs (of 8) evaluated on the FMA pipe (0, 1 and 2 within 1 %)
 
 template <int D>
 struct AttnCfg {
@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // columns [64, 128): those of S columns [64, 128) (in registers) go to
         // [96, 128), then S columns [0, 64) are read again and theirs go to
         // [64, 96) -- every column written has been read already.  Packed
-        // fp32x2 math; 2 of every 8 exponential pairs on the FMA pipe.
+        // fp32x2 math; kAttnPolyOf8 of every 8 exponential pairs on the FMA pipe.
         const float2 c2v = f2(p.c2, p.c2), nm = f2(-m, -m);
         float2 acc2 = f2(0.f, 0.f);
         auto exp64 = [&](const uint32_t (&a0)[32], const uint32_t (&a1)[32], uint32_t (&pk)[32]) {

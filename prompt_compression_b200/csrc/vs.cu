@@ -50,7 +50,7 @@ constexpr int kVsProducerWarp = 8;
 constexpr int kVsMmaWarp = 9;
 constexpr int kVsThreads = 10 * 32;
 constexpr float kVsRescale = 8.f;
-constexpr int kVsPolyOf8 = 2;          // exponential pairs (of 8) evaluated on the FMA pipe
+constexpr int kVsPolyOf8 = 0;          // exponential pairs (of 8) on the FMA pipe: none (the kernel is ALU bound; measured best)
 
 template <int D>
 struct VsCfg {
@@ -520,11 +520,11 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         // P = 2^(c2 s - m) into TMEM columns [64, 128) of the S buffer: S
         // columns [64, 128) are read again and theirs go to [96, 128), then
         // those of S columns [0, 64) to [64, 96) -- every column written has
-        // been read.  Masked keys (s = -inf) give 0; a row
-        // that has seen no key yet (m = -inf) has only masked keys here (the
-        // FMA-pipe exponential turns a masked key into 2^-126 instead of 0:
-        // far below the rounding of the sum and of O, and wiped by the
-        // rescale when the row sees its first key).
+        // been read.  Masked keys (s = -inf) give 0; a row that has seen no
+        // key yet (m = -inf) has only masked keys here (with kVsPolyOf8 > 0
+        // the FMA-pipe exponential would turn a masked key into 2^-126
+        // instead of 0: far below the rounding of the sum and of O, and
+        // wiped by the rescale when the row sees its first key).
         const float mm = m == -INFINITY ? 0.f : m;
         const float2 c2v = f2(p.c2, p.c2), nm = f2(-mm, -mm);
         float2 acc2 = f2(0.f, 0.f);
