@@ -275,7 +275,10 @@ spk_status specpc_colsum(const spk_specpc_shape* shape, const void* q_bf16, cons
  * The pages say "local pooling" without its kind; the workloads use max
  * pooling, which is what topk_select does.  topk_select_pool takes the mode.
  * Workspace: units * round_up(n_cand, 4) * 4 bytes, 16-byte aligned (the
- * order-preserving 32-bit keys of the pooled values, one padded row per unit).
+ * order-preserving 32-bit keys of the pooled values, one padded row per
+ * unit).  It is required by the contract; rows of up to 327,680 candidates
+ * with pool_kernel <= 2049 keep their keys in shared memory instead and
+ * leave it untouched.
  *
  * Supported: pool_kernel odd >= 1; k >= 0; n_tail >= 0; n_cand >= 0;
  * pool_mode SPK_POOL_MAX or SPK_POOL_AVG.
