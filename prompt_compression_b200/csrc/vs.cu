@@ -462,17 +462,20 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         tc_fence_after();
         // S columns [0, 64) then [64, 128), masked: the row max
         // (a word every lane sees whole -- the common case in vertical
-        // tiles -- needs no select)
-        auto mask64 = [&](uint32_t (&a0)[32], uint32_t (&a1)[32], uint32_t v0, uint32_t v1) {
+        // tiles -- needs no select).  A masked word goes back to TMEM, so
+        // the second pass over S reads it masked.
+        auto mask64 = [&](uint32_t (&a0)[32], uint32_t (&a1)[32], uint32_t v0, uint32_t v1, uint32_t col) {
           if (__any_sync(0xffffffffu, v0 != 0xffffffffu)) {
 #pragma unroll
             for (int k = 0; k < 32; ++k)
               if (!((v0 >> k) & 1u)) a0[k] = __float_as_uint(-INFINITY);
+            vs_tmem_st32(col, a0);
           }
           if (__any_sync(0xffffffffu, v1 != 0xffffffffu)) {
 #pragma unroll
             for (int k = 0; k < 32; ++k)
               if (!((v1 >> k) & 1u)) a1[k] = __float_as_uint(-INFINITY);
+            vs_tmem_st32(col + 32, a1);
           }
         };
         auto max64 = [&](const uint32_t (&a0)[32], const uint32_t (&a1)[32], float mx) {
@@ -492,9 +495,10 @@ __global__ void __launch_bounds__(kVsThreads, 1)
           tmem_ld32(tlane + 64 * hh, a0);
           tmem_ld32(tlane + 64 * hh + 32, a1);
           tmem_ld_wait2(a0, a1);
-          mask64(a0, a1, hh ? vis[2] : vis[0], hh ? vis[3] : vis[1]);
+          mask64(a0, a1, hh ? vis[2] : vis[0], hh ? vis[3] : vis[1], tlane + 64 * hh);
           mx = max64(a0, a1, mx);
         }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");   // the masked words have landed
         const float mt = mx * p.c2;
         const bool need = mx != -INFINITY && mt > m + kVsRescale;
         if (__any_sync(0xffffffffu, need)) {
@@ -546,8 +550,7 @@ __global__ void __launch_bounds__(kVsThreads, 1)
           tmem_ld32(tlane + 64 * hh, a0);
           tmem_ld32(tlane + 64 * hh + 32, a1);
           tmem_ld_wait2(a0, a1);
-          mask64(a0, a1, hh ? vis[2] : vis[0], hh ? vis[3] : vis[1]);
-          exp32(a0, tlane + 64 + 32 * hh);
+          exp32(a0, tlane + 64 + 32 * hh);                // masked by the first pass
           exp32(a1, tlane + 64 + 32 * hh + 16);
         }
         l += acc2.x + acc2.y;
