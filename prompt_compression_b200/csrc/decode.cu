@@ -293,8 +293,8 @@ __global__ void __launch_bounds__(kDecMaxWarps * 32, 1)
 }
 
 // Persistent streaming over units, for short caches (up to 4 blocks of 16
-// rows per warp and unit): one CTA per SM takes the units blockIdx.x,
-// + gridDim.x, ...; warp w takes the 16-row blocks w, w + W, ... of each,
+// rows per warp and unit): one or two CTAs per SM take the units
+// blockIdx.x, + gridDim.x, ...; warp w takes the 16-row blocks w, w + W, ... of each,
 // and its two slots keep the next block in flight across unit boundaries, so
 // the loads of the next unit overlap the merge of the current one (the merge
 // state has its own shared memory).  Q fragments of the next unit are
@@ -471,11 +471,21 @@ cudaError_t launch_stream(const void* q, const void* k, const void* v, float* ou
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
+  // Up to 4 block positions per warp.  With at most 5 warps (20 blocks) two
+  // CTAs share an SM (their per-unit merges overlap each other's loads);
+  // otherwise up to kStreamMaxWarps warps, one CTA per SM.
   const int blocks = (n_kv + kStreamRows - 1) / kStreamRows;
-  const int per = (blocks + kStreamMaxWarps - 1) / kStreamMaxWarps;   // block positions per warp
+  constexpr int kPairWarps = 5;
+  int per = (blocks + kPairWarps - 1) / kPairWarps;                 // block positions per warp
+  int ctas_per_sm = 2;
+  if (per > 4) {
+    per = (blocks + kStreamMaxWarps - 1) / kStreamMaxWarps;
+    ctas_per_sm = 1;
+  }
   const int warps = (blocks + per - 1) / per;
   const int smem = warps * (2 * kSlotB + 8 * D * 4);
-  const int grid = units < sms ? units : sms;
+  static_assert(2 * kPairWarps * (2 * kSlotB + 8 * D * 4) <= 227 * 1024, "two CTAs of five warps share an SM");
+  const int grid = units < ctas_per_sm * sms ? units : ctas_per_sm * sms;
   decode_stream_kernel<D><<<grid, warps * 32, smem, stream>>>(static_cast<const uint16_t*>(q),
                                                               static_cast<const uint16_t*>(k),
                                                               static_cast<const uint16_t*>(v), out, units, g, n_kv,
