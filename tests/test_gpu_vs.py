@@ -89,6 +89,7 @@ def _inputs(seed, B, L, hq, hkv, d, n, n_q):
     (4, 1, 1, 4, 1, 128, 600, 257, 40, 0),      # no slash beyond the token itself
     (5, 2, 1, 2, 1, 128, 2000, 256, 200, 64),   # far vertical keys and diagonals
     (6, 1, 2, 6, 2, 128, 800, 300, 40, 12),     # g = 3: the second pair has one head
+    (7, 1, 1, 4, 2, 128, 65536, 200, 4096, 100),  # the largest pattern: n = 65536, 4096 vertical keys
 ])
 def test_vs_attention_parity(P, case):
     seed, B, L, hq, hkv, d, n, n_q, n_v, n_s = case
