@@ -12,10 +12,11 @@
 // later level counting only the keys that match the prefix found so far),
 // and the selection {key > T} u {the first take_eq keys == T} is emitted in
 // ascending index order: warps own contiguous, 128-key-aligned shares of the
-// row, one walk counts their keys above and equal to T, a prefix over warps
-// (and CTAs) gives each its output offset and its share of the ties (lowest
-// index first), and a second walk writes the indices.  No sort and no list:
-// any k, deterministic, ties to the lower index.
+// row and count their keys above and equal to T (one walk, or the last
+// histogram level's sweep in the cluster kernel), a prefix over warps (and
+// CTAs) gives each its output offset and its share of the ties (lowest index
+// first), and a walk writes the indices.  No sort and no list: any k,
+// deterministic, ties to the lower index.
 //
 // Two kernels do this.  topk_cluster_kernel (rows up to 8 x kSegMax
 // candidates, pooling radius up to kTile / 2) splits a row over a cluster of
