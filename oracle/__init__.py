@@ -194,7 +194,7 @@ def decode_attention(q, k, v, scale: float = 1.0):
     return out
 
 
-def prefill_unit(q, k, v, n_window: int, n_lookahead: int, n_in: int, scale: float = 1.0):
+def prefill_unit(q, k, v, n_window: int, n_lookahead: int, n_in: int, scale: float = 1.0, rows=None):
     """Prefill attention of one unit's window and lookahead rows.
 
     q [g, R, d] (R = n_window + n_lookahead), k/v [n_in + n_lookahead, d]
@@ -202,34 +202,38 @@ def prefill_unit(q, k, v, n_window: int, n_lookahead: int, n_in: int, scale: flo
     row i sits at position n_in - n_window + i, lookahead row i at
     n_in + (i - n_window); each attends to the keys up to its position.
     Returns (out [g, R, d] float64, lse_in [g * R], natural log over the
-    input keys only)."""
+    input keys only).  With rows = [(h, i), ...] only those rows are
+    evaluated and the result is (out [len(rows), d], lse_in [len(rows)])."""
     lib = _load()
     q = np.ascontiguousarray(q, np.uint16)
     k = np.ascontiguousarray(k, np.uint16)
     v = np.ascontiguousarray(v, np.uint16)
     g, R, d = q.shape
     assert R == n_window + n_lookahead and k.shape == v.shape and k.shape[0] >= n_in + n_lookahead
-    out = np.zeros((g, R, d), np.float64)
-    lse = np.zeros(g * R, np.float64)
-    for h in range(g):
-        for i in range(R):
-            pos = n_in - n_window + i if i < n_window else n_in + (i - n_window)
-            row = np.zeros(d, np.float64)
-            l = ctypes.c_double(0.0)
-            _check(lib.oracle_prefill_row(_ptr(q[h, i], _u16p), _ptr(k, _u16p), _ptr(v, _u16p), pos + 1, n_in, d,
-                                          scale, _ptr(row, _dp), ctypes.byref(l)))
-            out[h, i] = row
-            lse[h * R + i] = l.value
+    pairs = [(h, i) for h in range(g) for i in range(R)] if rows is None else [(int(h), int(i)) for h, i in rows]
+    out = np.zeros((len(pairs), d), np.float64)
+    lse = np.zeros(len(pairs), np.float64)
+    for j, (h, i) in enumerate(pairs):
+        assert 0 <= h < g and 0 <= i < R
+        pos = n_in - n_window + i if i < n_window else n_in + (i - n_window)
+        l = ctypes.c_double(0.0)
+        _check(lib.oracle_prefill_row(_ptr(q[h, i], _u16p), _ptr(k, _u16p), _ptr(v, _u16p), pos + 1, n_in, d,
+                                      scale, _ptr(out[j], _dp), ctypes.byref(l)))
+        lse[j] = l.value
+    if rows is None:
+        return out.reshape(g, R, d), lse
     return out, lse
 
 
-def vs_attention_unit(q, k, v, vertical, slash, scale: float = 1.0):
+def vs_attention_unit(q, k, v, vertical, slash, scale: float = 1.0, rows=None):
     """Vertical-Slash sparse attention of one unit's query heads.
 
     q [g, n_q, d]: the last n_q positions of the sequence (row i at
     n - n_q + i); k, v [n, d]; vertical: key indices every row sees; slash:
     offsets o = p - j every row sees (bf16 bit patterns for q, k, v).
-    Returns (out [g, n_q, d] float64, lse [g * n_q], natural log)."""
+    Returns (out [g, n_q, d] float64, lse [g * n_q], natural log).  With
+    rows = [(h, i), ...] only those rows are evaluated and the result is
+    (out [len(rows), d], lse [len(rows)])."""
     lib = _load()
     q = np.ascontiguousarray(q, np.uint16)
     k = np.ascontiguousarray(k, np.uint16)
@@ -240,16 +244,17 @@ def vs_attention_unit(q, k, v, vertical, slash, scale: float = 1.0):
     sm = np.zeros(n, np.uint8)
     vm[np.asarray(vertical, np.int64)] = 1
     sm[np.asarray(slash, np.int64)] = 1
-    out = np.zeros((g, n_q, d), np.float64)
-    lse = np.zeros(g * n_q, np.float64)
-    for h in range(g):
-        for i in range(n_q):
-            row = np.zeros(d, np.float64)
-            l = ctypes.c_double(0.0)
-            _check(lib.oracle_vs_row(_ptr(q[h, i], _u16p), _ptr(k, _u16p), _ptr(v, _u16p), _ptr(vm, _u8p),
-                                     _ptr(sm, _u8p), n, n - n_q + i, d, scale, _ptr(row, _dp), ctypes.byref(l)))
-            out[h, i] = row
-            lse[h * n_q + i] = l.value
+    pairs = [(h, i) for h in range(g) for i in range(n_q)] if rows is None else [(int(h), int(i)) for h, i in rows]
+    out = np.zeros((len(pairs), d), np.float64)
+    lse = np.zeros(len(pairs), np.float64)
+    for j, (h, i) in enumerate(pairs):
+        assert 0 <= h < g and 0 <= i < n_q
+        l = ctypes.c_double(0.0)
+        _check(lib.oracle_vs_row(_ptr(q[h, i], _u16p), _ptr(k, _u16p), _ptr(v, _u16p), _ptr(vm, _u8p),
+                                 _ptr(sm, _u8p), n, n - n_q + i, d, scale, _ptr(out[j], _dp), ctypes.byref(l)))
+        lse[j] = l.value
+    if rows is None:
+        return out.reshape(g, n_q, d), lse
     return out, lse
 
 

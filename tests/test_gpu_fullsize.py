@@ -164,3 +164,157 @@ def test_cascade_128k_full(P):
     ref = oracle.specpc_batch(bits_of(q1[0]), bits_of(k1[0]), W.specpc_row_weights(d.n_rows).astype(np.float32)
                               .astype(np.float64), 1, d.n_lookahead)
     assert_scores_close(s1[0].cpu().numpy(), ref, "specpc 128K one-layer scores")
+
+
+def _sample_rows(rng, g, R, extra=8, boundaries=()):
+    """(query head, row) pairs to check: the first and last row of every
+    query head, the given rows of head 0, and a few random ones."""
+    rows = {(h, 0) for h in range(g)} | {(h, R - 1) for h in range(g)}
+    rows |= {(0, i) for i in boundaries if 0 <= i < R}
+    target = len(rows) + extra
+    while len(rows) < target:
+        rows.add((int(rng.integers(g)), int(rng.integers(R))))
+    return sorted(rows)
+
+
+def test_prefill_attention_qwen32b_64k_full(P):
+    """The prefill attention of the window and lookahead rows at the 64K
+    workload, launched as the +prefill step launches it (every unit, the
+    column pass's workspace filled), then the column pass on its row offsets.
+    Sampled rows of sampled units against the fp64 oracle (output and
+    input-key LSE); every unit through properties (each output row is a
+    convex combination of V rows, every LSE finite, each row's attention mass
+    over the input keys is 1); the scores of a sampled unit against the
+    oracle."""
+    import torch
+    from prompt_compression_b200.pipeline import SpeckvBuffers
+    cfg = W.QWEN32B_64K
+    inp = W.speckv_inputs(cfg, seed=7, device="cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    gen = torch.Generator(device="cuda").manual_seed(24)
+    lshape = (cfg.batch, cfg.layers, cfg.hkv, cfg.n_lookahead, cfg.head_dim)
+    k_look = torch.randn(lshape, generator=gen, device="cuda").to(torch.bfloat16)
+    v_look = torch.randn(lshape, generator=gen, device="cuda").to(torch.bfloat16)
+    buf = SpeckvBuffers(q, k, v, cfg.n_window, cfg.c_max, window_mass=True)
+    g, R, nw, nl, n_in, d = cfg.g, cfg.rows, cfg.n_window, cfg.n_lookahead, cfg.n_in, cfg.head_dim
+    lse2 = torch.empty((cfg.units, g * R), dtype=torch.float32, device="cuda")
+    out = P.speckv_prefill_attention(q, k, v, k_look, v_look, nw, lse2=lse2, workspace=buf.ws_score)
+    P.speckv_colsum(q, k, nw, buf.scores, buf.ws_score, window_mass=buf.window_mass)
+    torch.cuda.synchronize()
+    assert P.spk_device_error() == (0, 0)
+
+    # ---- every unit
+    assert bool(torch.isfinite(lse2).all())
+    vmax = torch.maximum(v.view(cfg.units, -1).abs().amax(1), v_look.view(cfg.units, -1).abs().amax(1)).float()
+    omax = out.view(cfg.units, -1).abs().amax(1).float()
+    assert bool((omax <= vmax * (1 + 2.0 ** -8)).all()), (omax - vmax).max().item()
+    tot = buf.scores.double().sum(1) + buf.window_mass.double().sum(1)
+    assert torch.allclose(tot, torch.full_like(tot, g * R), rtol=1e-4, atol=0), tot.min().item()
+
+    # ---- sampled rows of sampled units against the oracle
+    rng = np.random.default_rng(1)
+    for u in (0, cfg.units - 1):
+        b, l, h = u // (cfg.layers * cfg.hkv), (u // cfg.hkv) % cfg.layers, u % cfg.hkv
+        qb = bits_of(q[b, l, h * g:(h + 1) * g])
+        kb = np.concatenate([bits_of(k[b, l, h]), bits_of(k_look[b, l, h])])
+        vb = np.concatenate([bits_of(v[b, l, h]), bits_of(v_look[b, l, h])])
+        rows = _sample_rows(rng, g, R, boundaries=(nw - 1, nw, 127, 128))
+        ref, rlse = oracle.prefill_unit(qb, kb, vb, nw, nl, n_in, rows=rows)
+        ob = W.bf16_decode(bits_of(out[b, l, h * g:(h + 1) * g])).astype(np.float64)
+        got = np.stack([ob[hh, i] for hh, i in rows])
+        bound = 2.0 ** -8 * np.abs(W.bf16_decode(vb)).max()
+        err = np.abs(got - ref).max()
+        assert err <= bound, f"unit {u}: out error {err:.3e} > {bound:.3e}"
+        lg = lse2[u].cpu().numpy()
+        np.testing.assert_allclose([lg[hh * R + i] for hh, i in rows], rlse / math.log(2.0), rtol=4e-7, atol=6e-5)
+    u = cfg.units - 1
+    b, l, h = u // (cfg.layers * cfg.hkv), (u // cfg.hkv) % cfg.layers, u % cfg.hkv
+    s, wm = oracle.speckv_unit(bits_of(q[b, l, h * g:(h + 1) * g]), bits_of(k[b, l, h]), nw, nl)
+    assert_scores_close(buf.scores[u].cpu().numpy(), s, f"scores from the prefill's row offsets, unit {u}")
+    assert_scores_close(buf.window_mass[u].cpu().numpy(), wm, f"window mass from the prefill, unit {u}")
+    del inp, q, k, v, k_look, v_look, buf, out
+    torch.cuda.empty_cache()
+
+
+def test_decode_qwen32b_compressed_full(P):
+    """Decode over the compressed cache at the benched shape (64 layers x 40
+    query heads over 320 kept rows per KV head): every output against the
+    oracle; then over the full 65,536-row cache, sampled layers against the
+    oracle (tolerance as in the decode parity tests: 1e-4 of max |v|)."""
+    import torch
+    cfg = W.DECODE_QWEN32B
+    B_, L, hq, hkv, d = cfg.batch, cfg.layers, cfg.hq, cfg.hkv, cfg.head_dim
+    gen = torch.Generator(device="cuda").manual_seed(5)
+
+    def rnd(*shape):
+        return torch.randn(shape, generator=gen, device="cuda").to(torch.bfloat16)
+
+    scale = d ** -0.5
+    q = rnd(B_, L, hq, d)
+    kc, vc = rnd(B_, L, hkv, cfg.n_kv, d), rnd(B_, L, hkv, cfg.n_kv, d)
+    out = torch.empty((B_, L, hq, d), dtype=torch.float32, device="cuda")
+    P.decode_attention(q, kc, vc, out, scale)
+    torch.cuda.synchronize()
+    assert P.spk_device_error() == (0, 0)
+    ref = oracle.decode_attention(bits_of(q), bits_of(kc), bits_of(vc), scale)
+    vmax = float(vc.abs().max())
+    np.testing.assert_allclose(out.cpu().numpy(), ref, rtol=0, atol=1e-4 * vmax)
+
+    kf, vf = rnd(B_, L, hkv, cfg.n_kv_full, d), rnd(B_, L, hkv, cfg.n_kv_full, d)
+    P.decode_attention(q, kf, vf, out, scale)
+    torch.cuda.synchronize()
+    assert P.spk_device_error() == (0, 0)
+    for l in (0, L - 1):
+        ref = oracle.decode_attention(bits_of(q[:, l:l + 1]), bits_of(kf[:, l:l + 1]), bits_of(vf[:, l:l + 1]),
+                                      scale)
+        vmax = float(vf[:, l].abs().max())
+        np.testing.assert_allclose(out[:, l:l + 1].cpu().numpy(), ref, rtol=0, atol=1e-4 * vmax)
+    del kf, vf
+    torch.cuda.empty_cache()
+
+
+def test_vs_llama8b_16k_full(P):
+    """Vertical-Slash sparse prefill at the benched workload (32 layers, every
+    one of the 16,384 rows, 1024 vertical keys and 80 diagonals per unit):
+    sampled rows of sampled units against the fp64 oracle (output within
+    2^-8 of max |v|, LSE as in the Vertical-Slash parity tests), every unit
+    through properties (outputs convex combinations of V rows, LSE finite)."""
+    import torch
+    cfg = W.VS_LLAMA8B_16K
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    shape_q = (cfg.batch, cfg.layers, cfg.hq, cfg.n_q, cfg.head_dim)
+    shape_k = (cfg.batch, cfg.layers, cfg.hkv, cfg.n, cfg.head_dim)
+    q = (torch.randn(shape_q, generator=gen, device="cuda") / cfg.head_dim ** 0.5).to(torch.bfloat16)
+    k = torch.randn(shape_k, generator=gen, device="cuda").to(torch.bfloat16)
+    v = torch.randn(shape_k, generator=gen, device="cuda").to(torch.bfloat16)
+    vert, sl = W.vs_pattern(cfg, seed=9, device="cuda")
+    ws = torch.empty(P.vs_workspace_size(P.binding.vs_shape(q, k, cfg.n_vertical, cfg.n_slash)), dtype=torch.uint8,
+                     device="cuda")
+    lse2 = torch.empty((cfg.batch * cfg.layers * cfg.hq, cfg.n_q), dtype=torch.float32, device="cuda")
+    out = P.vs_sparse_attention(q, k, v, vert, sl, lse2=lse2, workspace=ws)
+    torch.cuda.synchronize()
+    assert P.spk_device_error() == (0, 0)
+
+    g = cfg.g
+    assert bool(torch.isfinite(lse2).all())
+    vmax = v.view(cfg.units, -1).abs().amax(1).float()
+    omax = out.view(cfg.units, -1).abs().amax(1).float()
+    assert bool((omax <= vmax * (1 + 2.0 ** -8)).all()), (omax - vmax).max().item()
+
+    rng = np.random.default_rng(2)
+    vert_c, sl_c = vert.cpu().numpy(), sl.cpu().numpy()
+    for u in (0, cfg.units // 2 + 1, cfg.units - 1):
+        b, l, h = u // (cfg.layers * cfg.hkv), (u // cfg.hkv) % cfg.layers, u % cfg.hkv
+        qb = bits_of(q[b, l, h * g:(h + 1) * g])
+        kb, vb = bits_of(k[b, l, h]), bits_of(v[b, l, h])
+        rows = _sample_rows(rng, g, cfg.n_q, extra=12, boundaries=(1, 127, 128, 8191, 8192))
+        ref, rlse = oracle.vs_attention_unit(qb, kb, vb, vert_c[u], sl_c[u], rows=rows)
+        ob = W.bf16_decode(bits_of(out[b, l, h * g:(h + 1) * g])).astype(np.float64)
+        got = np.stack([ob[hh, i] for hh, i in rows])
+        bound = 2.0 ** -8 * np.abs(W.bf16_decode(vb)).max()
+        err = np.abs(got - ref).max()
+        assert err <= bound, f"unit {u}: out error {err:.3e} > {bound:.3e}"
+        lg = lse2[u * g:(u + 1) * g].cpu().numpy()
+        np.testing.assert_allclose([lg[hh, i] for hh, i in rows], rlse / math.log(2.0), rtol=4e-7, atol=6e-5)
+    del q, k, v, out, lse2, ws
+    torch.cuda.empty_cache()

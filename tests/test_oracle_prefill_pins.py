@@ -47,6 +47,23 @@ def test_prefill_matches_bruteforce_attention(g, nw, nl, n_in, d):
             np.testing.assert_allclose(lse[h * R + i], logsumexp(z[:min(pos + 1, n_in)]), rtol=1e-13)
 
 
+def test_prefill_sampled_rows_match_bruteforce():
+    # the row-sampling form (used at full sizes) evaluates exactly the asked
+    # rows, in the asked order, each equal to the literal attention row
+    g, nw, nl, n_in, d = 3, 9, 6, 80, 8
+    rng = np.random.default_rng(31)
+    q, k, v = _case(rng, g, nw, nl, n_in, d)
+    rows = [(2, 14), (0, 0), (1, 8), (1, 9), (2, 0), (0, 14)]
+    out, lse = oracle.prefill_unit(q, k, v, nw, nl, n_in, scale=0.9, rows=rows)
+    assert out.shape == (len(rows), d) and lse.shape == (len(rows),)
+    Q, K, V = _vals(q), _vals(k), _vals(v)
+    for j, (h, i) in enumerate(rows):
+        pos = n_in - nw + i if i < nw else n_in + i - nw
+        z = 0.9 * K[:pos + 1] @ Q[h, i]
+        np.testing.assert_allclose(out[j], softmax(z) @ V[:pos + 1], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(lse[j], logsumexp(z[:min(pos + 1, n_in)]), rtol=1e-13)
+
+
 def test_prefill_closed_forms():
     d = 8
     rng = np.random.default_rng(5)

@@ -57,6 +57,22 @@ def test_vs_matches_masked_bruteforce(g, n_q, n, d, nv, ns):
     np.testing.assert_allclose(lse, rlse, rtol=1e-13)
 
 
+def test_vs_sampled_rows_match_bruteforce():
+    # the row-sampling form (used at full sizes) evaluates exactly the asked
+    # rows, in the asked order
+    g, n_q, n, d = 2, 30, 70, 8
+    rng = np.random.default_rng(77)
+    q, k, v = _case(rng, g, n_q, n, d)
+    vert = np.sort(rng.choice(n, size=9, replace=False))
+    sl = np.sort(rng.choice(n, size=5, replace=False))
+    rows = [(1, 29), (0, 0), (1, 3), (0, 17)]
+    out, lse = oracle.vs_attention_unit(q, k, v, vert, sl, scale=0.8, rows=rows)
+    ref, rlse = _bruteforce(q, k, v, vert, sl, 0.8)
+    for j, (h, i) in enumerate(rows):
+        np.testing.assert_allclose(out[j], ref[h, i], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(lse[j], rlse[h * n_q + i], rtol=1e-13)
+
+
 def test_vs_full_pattern_is_dense_causal_attention():
     # every key vertical, or every offset a slash: plain causal attention,
     # which is the oracle's (pinned) prefill attention with no lookahead
