@@ -104,31 +104,57 @@ __device__ __forceinline__ uint32_t vs_pack_bf16(float lo, float hi) {
 __device__ __forceinline__ int vs_site(int role, int which) { return 400 + role * 10 + which; }
 
 
-// The next slash tile of an item, walking down from tile t: tile t is crossed
-// iff some offset o in S u {0} lies in [p0 - 128 t - 127, p_last - 128 t].
-// a indexes the first offset of S (ascending) not below the window's lower
-// end, which only grows as t falls.  Returns -1 when no tile is left.
-__device__ __forceinline__ int next_slash_tile(const int* __restrict__ S, int n_s, int p0, int p_last, int& t,
-                                               int& a) {
-  while (t >= 0) {
-    const int lo = p0 - 128 * t - 127, hi = p_last - 128 * t;
-    while (a < n_s && __ldg(S + a) < lo) ++a;
-    const bool hit = (lo <= 0 && 0 <= hi) || (a < n_s && __ldg(S + a) <= hi);
-    const int cur = t--;
-    if (hit) return cur;
+// Marks in `tb` (one bit per 128-key tile) the slash tiles of an item whose
+// rows sit at positions p0 .. p_last (p_last - p0 < 128): tile t (0 <= t <=
+// p_last / 128) is crossed iff some offset o in S u {0} lies in
+// [p0 - 128 t - 127, p_last - 128 t], i.e. t in [floor((p0 - o) / 128),
+// floor((p_last - o) / 128)] -- at most two tiles per offset.  Thread `tid`
+// of `nthreads` takes every nthreads-th offset (the loads are independent);
+// the caller clears the words first and synchronises after.
+__device__ __forceinline__ void mark_slash_tiles(uint32_t* tb, const int* __restrict__ S, int n_s, int p0, int p_last,
+                                                 int tid, int nthreads) {
+  const int t_top = p_last >> 7;
+  for (int i = tid; i <= n_s; i += nthreads) {
+    const int o = i < n_s ? __ldg(S + i) : 0;
+    const int lo = max((p0 - o) >> 7, 0), hi = min((p_last - o) >> 7, t_top);
+    for (int t = lo; t <= hi; ++t) atomicOr(&tb[t >> 5], 1u << (t & 31));
   }
-  return -1;
 }
 
-// Number of entries of the ascending array x[0, n) that are <= v.
-__device__ __forceinline__ int upper_bound_le_global(const int* __restrict__ x, int n, int v) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(x + mid) <= v) lo = mid + 1;
-    else hi = mid;
+// Walks the set bits of a tile bitmap from the highest down (the order in
+// which every role takes an item's slash tiles).
+struct TileWalk {
+  int w;
+  uint32_t m;
+  __device__ __forceinline__ TileWalk(const uint32_t* tb, int t_top) : w(t_top >> 5), m(tb[t_top >> 5]) {}
+  __device__ __forceinline__ int next(const uint32_t* tb) {
+    while (m == 0u) {
+      if (--w < 0) return -1;
+      m = tb[w];
+    }
+    const int b = 31 - __clz(m);
+    m &= ~(1u << b);
+    return w * 32 + b;
   }
-  return lo;
+};
+
+// Number of entries of the ascending array x[0, n) that are <= v, by the
+// whole warp: 32 probes per step narrow the answer's range 32-fold, so
+// n <= 32^k takes k dependent loads.  Every lane returns the count.
+__device__ __forceinline__ int warp_count_le(const int* __restrict__ x, int n, int v, int lane) {
+  int lo = 0, len = n;                  // the count lies in [lo, lo + len]
+  while (len > 32) {
+    const int step = (len + 31) >> 5;
+    const int i = lo + lane * step;
+    const bool le = i < lo + len && __ldg(x + i) <= v;
+    const int c = __popc(__ballot_sync(0xffffffffu, le));   // probes <= v: a prefix
+    if (c == 0) return lo;
+    const int nlo = lo + (c - 1) * step + 1;
+    len = min(lo + c * step, lo + len) - nlo;
+    lo = nlo;
+  }
+  const bool le = lane < len && __ldg(x + lo + lane) <= v;
+  return lo + __popc(__ballot_sync(0xffffffffu, le));
 }
 
 // 32 bits of a bitmap starting at bit o (bits below 0 and at or above
@@ -163,7 +189,9 @@ __global__ void __launch_bounds__(kVsThreads, 1)
   // per Q tile x (0: A, 1: B): s_full[x], p_full[x] (4 warps), pv_done[x], o_empty[x] (4 warps)
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
       p_full[2], pv_done[2], o_empty[2], done_bar, soft_bar;
-  __shared__ uint32_t slash_tiles[kVsMaxN / 128 / 32];   // tiles of the current item that were slash tiles
+  __shared__ uint32_t slash_tiles[kVsMaxN / 128 / 32];   // the softmax warps' item: its slash tiles
+  __shared__ uint32_t prod_tiles[kVsMaxN / 128 / 32];    // the producer's item
+  __shared__ uint32_t mma_tiles[kVsMaxN / 128 / 32];     // the UMMA issuer's item
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
 
@@ -217,13 +245,18 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     p0 = n - p.n_q + rb * 128;
     p_last = n - p.n_q + min(rb * 128 + 127, p.n_q - 1);
   };
-  // tiles of an item: its slash tiles, then ceil(cv / 128) vertical tiles
-  auto count_tiles = [&](int u, int p0, int p_last, int& n_slash, int& cv) {
-    const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
-    int t = p_last >> 7, a = 0;
+  // tiles of an item: its slash tiles (marked in tb), then ceil(cv / 128)
+  // vertical tiles (cv = vertical keys <= p_last); whole warp, every lane
+  // returns the counts
+  auto warp_item_tiles = [&](uint32_t* tb, int u, int p0, int p_last, int& n_slash, int& cv) {
+    const int nw = ((p_last >> 7) >> 5) + 1;
+    for (int w = lane; w < nw; w += 32) tb[w] = 0u;
+    __syncwarp();
+    mark_slash_tiles(tb, p.slash + static_cast<size_t>(u) * p.n_s, p.n_s, p0, p_last, lane, 32);
+    __syncwarp();
     n_slash = 0;
-    while (next_slash_tile(S, p.n_s, p0, p_last, t, a) >= 0) ++n_slash;
-    cv = p.n_v > 0 ? upper_bound_le_global(p.vert + static_cast<size_t>(u) * p.n_v, p.n_v, p_last) : 0;
+    for (int w = 0; w < nw; ++w) n_slash += __popc(tb[w]);
+    cv = p.n_v > 0 ? warp_count_le(p.vert + static_cast<size_t>(u) * p.n_v, p.n_v, p_last, lane) : 0;
     return n_slash + (cv + 127) / 128;
   };
 
@@ -231,7 +264,8 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     // (no other warps)
   } else if (warp == kVsProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // (the whole warp derives each item's tiles; lane 0 issues the copies)
+    {
       bool ok = true;
       uint32_t tile_count = 0;
       int items_done = 0;
@@ -240,7 +274,8 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         int u, hp, rb, p0, p_last;
         item_geom(item, u, hp, rb, p0, p_last);
         int n_slash, cv;
-        const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
+        const int n_tiles = warp_item_tiles(prod_tiles, u, p0, p_last, n_slash, cv);
+        if (lane == 0) do {
         if (!(ok = mbar_wait(&q_empty, (items_done & 1) ^ 1, abort_v, vs_site(0, 0)))) break;
         mbar_arrive_expect_tx(&q_full, 2 * C::kTileBytes);
         for (int x = 0; x < 2; ++x) {
@@ -250,13 +285,12 @@ __global__ void __launch_bounds__(kVsThreads, 1)
             tma_load_3d(Q_s + x * C::kTileBytes + a * 16384, &qmap, &q_full, a * 64, rb * 128, qh);
         }
         q_last = items_done & 1;
-        const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
-        int t = p_last >> 7, sa = 0;
+        TileWalk walk(prod_tiles, p_last >> 7);
         for (int i = 0; ok && i < n_tiles; ++i, ++tile_count) {
           const int st = tile_count & 1;
           const uint32_t ph = (tile_count >> 1) & 1;
           const bool slash = i < n_slash;
-          const int row0 = slash ? 128 * next_slash_tile(S, p.n_s, p0, p_last, t, sa) : 128 * (i - n_slash);
+          const int row0 = slash ? 128 * walk.next(prod_tiles) : 128 * (i - n_slash);
           if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, abort_v, vs_site(0, 1)))) break;
           mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
           for (int a = 0; a < C::kAtoms; ++a)
@@ -268,8 +302,10 @@ __global__ void __launch_bounds__(kVsThreads, 1)
             tma_load_3d(V_s + st * C::kTileBytes + a * 16384, slash ? &vmap : &vvmap, &v_full[st], a * 64, row0, u);
           v_last[st] = static_cast<int>(ph);
         }
+        } while (false);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
-      if (!ok) {
+      if (lane == 0 && !ok) {
         volatile int never = 0;
         if (q_last >= 0) mbar_wait(&q_full, q_last, &never, vs_site(0, 7), 100000000ull);
         for (int s = 0; s < 2; ++s) {
@@ -283,7 +319,8 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     // Order per key tile t: O_A += P_A V(t), S_A(t+1), O_B += P_B V(t), S_B(t+1)
     // (each softmax group works while the other's products run; S_x(t+1)
     // follows O_x's product of tile t, so O_x is quiescent once it lands).
-    if (lane == 0) {
+    // (the whole warp derives each item's tile count; lane 0 issues)
+    {
       bool ok = true;
       uint32_t T = 0;
       int items_done = 0;
@@ -329,23 +366,28 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         int u, hp, rb, p0, p_last;
         item_geom(item, u, hp, rb, p0, p_last);
         int n_slash, cv;
-        const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
-        if (!(ok = mbar_wait(&q_full, items_done & 1, abort_v, vs_site(1, 0)))) break;
-        if (!(ok = issue_s(0, T)) || !(ok = issue_s(1, T))) break;
-        for (int t = 0; ok && t < n_tiles; ++t) {
-          const uint32_t Tc = T + t;
-          if (!(ok = issue_pv(0, Tc, t))) break;
-          if (t + 1 < n_tiles && !(ok = issue_s(0, Tc + 1))) break;
-          if (!(ok = issue_pv(1, Tc, t))) break;
-          if (t + 1 < n_tiles && !(ok = issue_s(1, Tc + 1))) break;
-        }
-        if (!ok) break;
-        umma_commit(&q_empty);
+        const int n_tiles = warp_item_tiles(mma_tiles, u, p0, p_last, n_slash, cv);
+        if (lane == 0) do {
+          if (!(ok = mbar_wait(&q_full, items_done & 1, abort_v, vs_site(1, 0)))) break;
+          if (!(ok = issue_s(0, T)) || !(ok = issue_s(1, T))) break;
+          for (int t = 0; ok && t < n_tiles; ++t) {
+            const uint32_t Tc = T + t;
+            if (!(ok = issue_pv(0, Tc, t))) break;
+            if (t + 1 < n_tiles && !(ok = issue_s(0, Tc + 1))) break;
+            if (!(ok = issue_pv(1, Tc, t))) break;
+            if (t + 1 < n_tiles && !(ok = issue_s(1, Tc + 1))) break;
+          }
+          if (!ok) break;
+          umma_commit(&q_empty);
+        } while (false);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         T += n_tiles;
       }
-      umma_commit(&done_bar);
-      volatile int never = 0;
-      mbar_wait(&done_bar, 0, &never, vs_site(1, 9), 100000000ull);
+      if (lane == 0) {
+        umma_commit(&done_bar);
+        volatile int never = 0;
+        mbar_wait(&done_bar, 0, &never, vs_site(1, 9), 100000000ull);
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax groups
@@ -374,13 +416,17 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++items_done) {
       int u, hp, rb, p0, p_last;
       item_geom(item, u, hp, rb, p0, p_last);
-      int n_slash, cv;
-      const int n_tiles = count_tiles(u, p0, p_last, n_slash, cv);
-      // this unit's pattern as bitmaps (and V as a list), and no slash tile yet
+      // this unit's pattern as bitmaps (and V as a list), and the item's
+      // slash tiles as a bitmap
       if (!(ok = softmax_sync())) break;                // the previous item is done with them
-      if (u != loaded_unit) {
+      const int tb_words = ((p_last >> 7) >> 5) + 1;
+      for (int w = tid; w < tb_words; w += 256) slash_tiles[w] = 0u;
+      const bool new_unit = u != loaded_unit;
+      if (new_unit)
         for (int w = tid; w < n_words; w += 256) { vbits[w] = 0u; sbits[w] = 0u; }
-        if (!(ok = softmax_sync())) break;
+      if (!(ok = softmax_sync())) break;
+      mark_slash_tiles(slash_tiles, p.slash + static_cast<size_t>(u) * p.n_s, p.n_s, p0, p_last, tid, 256);
+      if (new_unit) {
         const int* vg = p.vert + static_cast<size_t>(u) * p.n_v;
         const int* sg = p.slash + static_cast<size_t>(u) * p.n_s;
         for (int i = tid; i < p.n_v; i += 256) {
@@ -396,25 +442,25 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         }
         loaded_unit = u;
       }
-      for (int w = tid; w < kVsMaxN / 128 / 32; w += 256) slash_tiles[w] = 0u;
       if (!(ok = softmax_sync())) break;
+      int n_slash = 0;
+      for (int w = 0; w < tb_words; ++w) n_slash += __popc(slash_tiles[w]);
+      const int cv = p.n_v > 0 ? warp_count_le(p.vert + static_cast<size_t>(u) * p.n_v, p.n_v, p_last, lane) : 0;
+      const int n_tiles = n_slash + (cv + 127) / 128;
 
       const int h = 2 * hp + x;                         // head of the group
       const int qh = u * p.g + h;
       const int i_row = rb * 128 + r;
       const bool live = i_row < p.n_q && h < p.g;
       const int pos = i_row < p.n_q ? n - p.n_q + i_row : n - 1;
-      const int* S = p.slash + static_cast<size_t>(u) * p.n_s;
-      int wt = p_last >> 7, wa = 0;                     // this role's walk over the slash tiles
+      TileWalk walk(slash_tiles, p_last >> 7);          // this role's walk over the slash tiles
       float m = -INFINITY, l = 0.f;
       for (int t = 0; ok && t < n_tiles; ++t) {
         const uint32_t Tc = T + t;
         const bool slash = t < n_slash;
         int j0 = 0;
         if (slash) {
-          const int tile = next_slash_tile(S, p.n_s, p0, p_last, wt, wa);
-          j0 = tile * 128;
-          if (lane == 0) atomicOr(&slash_tiles[tile >> 5], 1u << (tile & 31));   // read back by this warp only
+          j0 = walk.next(slash_tiles) * 128;
         }
         // visibility of the tile's 128 keys for this row, 32 per word
         uint32_t vis[4];
