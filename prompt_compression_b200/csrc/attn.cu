@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t T = 0;              // key tiles of this CTA before the current item
       int items_done = 0;
       const uint32_t idesc_s = idesc_bf16_f32(128, 128);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 64) | (1u << 16);   // B (V) MN-major
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D) | (1u << 16);    // B (V) MN-major, N = head_dim
       auto issue_s = [&](int x, uint32_t Ti) -> bool {
         const int st = Ti & 1;
         if (x == 0 && !mbar_wait(&k_full[st], (Ti >> 1) & 1, abort_v, attn_site(1, 1))) return false;
@@ -257,12 +257,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t v_base = smem_u32(V_s + st * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-          for (int a = 0; a < C::kAtoms; ++a) {
-            const uint64_t v_desc = sw128_mnmajor_desc(v_base + a * 16384 + kk * 2048, 16384);
-            umma_bf16_ts(tmem_base + x * 256 + 128 + a * 64, tmem_base + x * 256 + 64 + kk * 8, v_desc, idesc_pv,
-                         (t > 0 || kk > 0) ? 1u : 0u);
-          }
+          // one instruction spans the head_dim / 64 column blocks (lbo apart)
+          const uint64_t v_desc = sw128_mnmajor_desc(v_base + kk * 2048, 16384);
+          umma_bf16_ts(tmem_base + x * 256 + 128, tmem_base + x * 256 + 64 + kk * 8, v_desc, idesc_pv,
+                       (t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[x]);
         if (x == 1) umma_commit(&v_empty[st]);
