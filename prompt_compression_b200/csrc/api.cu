@@ -15,6 +15,8 @@
 #include "score.cuh"
 
 namespace spk {
+SPK_ERROR_READER(device_errors_api)
+
 // decode.cu
 cudaError_t launch_decode(const void* q, const void* k, const void* v, float* out, int units, int g,
                           int head_dim, int n_kv, float c2, cudaStream_t stream);
@@ -630,17 +632,18 @@ spk_status spk_mapped_host_pointer(const void* host, void** dev) {
 spk_status spk_device_error(int* status, int* site, int clear) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  // every translation unit's error word, the first set one in this order
+  // reported (the others are cleared with it)
+  cudaError_t (*const readers[])(int*, int*, bool) = {device_errors_api, device_errors_score, device_errors_attn,
+                                                       device_errors_vs, device_errors_compact};
   int code = 0, where = 0;
-  if ((e = cudaMemcpyFromSymbol(&code, g_device_error, sizeof code)) != cudaSuccess)
-    return cuda_fail(e, "reading the device error word");
-  if ((e = cudaMemcpyFromSymbol(&where, g_device_error_site, sizeof where)) != cudaSuccess)
-    return cuda_fail(e, "reading the device error site");
-  if (clear) {
-    const int zero = 0;
-    if ((e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero)) != cudaSuccess)
-      return cuda_fail(e, "clearing the device error word");
-    if ((e = cudaMemcpyToSymbol(g_device_error_site, &zero, sizeof zero)) != cudaSuccess)
-      return cuda_fail(e, "clearing the device error site");
+  for (auto rd : readers) {
+    int c = 0, w = 0;
+    if ((e = rd(&c, &w, clear != 0)) != cudaSuccess) return cuda_fail(e, "reading a device error word");
+    if (code == 0 && c != 0) {
+      code = c;
+      where = w;
+    }
   }
   if (status) *status = code == SPK_DEVERR_NONE ? SPK_OK : (code == SPK_DEVERR_TIMEOUT ? SPK_ERR_TIMEOUT : SPK_ERR_ARG);
   if (site) *site = where;

@@ -47,6 +47,9 @@
 #include "score.cuh"
 
 namespace spk {
+
+SPK_ERROR_READER(device_errors_attn)
+
 namespace {
 
 constexpr int kAttnSoftmaxWarps = 4;     // per Q tile; two groups

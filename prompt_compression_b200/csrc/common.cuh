@@ -23,8 +23,26 @@ enum DeviceError : int {
   SPK_DEVERR_INDEX = 2,        // kv_compact saw an index outside [0, n_src)
 };
 
-extern __device__ int g_device_error;
-extern __device__ int g_device_error_site;
+// Each translation unit has its own error word (internal linkage: the
+// library is compiled without relocatable device code); a unit whose kernels
+// record errors defines its reader with SPK_ERROR_READER, and
+// spk_device_error() asks every reader.
+namespace {
+__device__ int g_device_error = 0;
+__device__ int g_device_error_site = 0;
+}  // namespace
+
+#define SPK_ERROR_READER(NAME)                                                                      \
+  cudaError_t NAME(int* code, int* site, bool clear) {                                              \
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_device_error, sizeof(int));                        \
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(site, g_device_error_site, sizeof(int));         \
+    if (e == cudaSuccess && clear) {                                                                \
+      const int zero = 0;                                                                           \
+      e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);                                   \
+      if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error_site, &zero, sizeof zero);        \
+    }                                                                                               \
+    return e;                                                                                       \
+  }
 
 #ifndef SPK_WAIT_LIMIT_NS
 #define SPK_WAIT_LIMIT_NS 2000000000ull   // 2 s: far above any legitimate pipeline stall

@@ -11,6 +11,9 @@
 #include "score.cuh"
 
 namespace spk {
+
+SPK_ERROR_READER(device_errors_compact)
+
 namespace {
 
 __global__ void __launch_bounds__(256)

@@ -43,8 +43,7 @@
 
 namespace spk {
 
-__device__ int g_device_error = 0;
-__device__ int g_device_error_site = 0;
+SPK_ERROR_READER(device_errors_score)
 
 namespace {
 

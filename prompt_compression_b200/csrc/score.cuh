@@ -69,6 +69,14 @@ struct ScoreParams {
 
 cudaError_t launch_score(int mode, int head_dim, const CUtensorMap& amap, const CUtensorMap& bmap,
                          const ScoreParams& p, int grid, cudaStream_t stream);
+
+// Device error words, one per translation unit that records errors (read,
+// and cleared when `clear`, by spk_device_error()).
+cudaError_t device_errors_api(int* code, int* site, bool clear);
+cudaError_t device_errors_score(int* code, int* site, bool clear);
+cudaError_t device_errors_attn(int* code, int* site, bool clear);
+cudaError_t device_errors_vs(int* code, int* site, bool clear);
+cudaError_t device_errors_compact(int* code, int* site, bool clear);
 // scores[b][j] = max_qh sum_g part[(b * n_blocks + j / 256) * groups + g][qh][j % 256]
 cudaError_t launch_specpc_merge(const float* part, int batch, int n_in, int n_blocks, int groups, int hq,
                                 float* scores, cudaStream_t stream);

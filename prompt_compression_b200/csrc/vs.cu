@@ -43,6 +43,9 @@
 #include "score.cuh"
 
 namespace spk {
+
+SPK_ERROR_READER(device_errors_vs)
+
 namespace {
 
 constexpr int kVsGroupWarps = 4;       // softmax warps per head of the pair (two groups)
