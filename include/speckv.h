@@ -26,7 +26,7 @@
  *     host and returned BEFORE anything is launched; spk_last_error() then
  *     describes the problem (thread-local string).
  *   - Errors found on the device (a bounded wait that timed out, an index
- *     outside its range in kv_compact) are recorded in a device error word
+ *     outside its range in kv_compact) are recorded in device error words
  *     that spk_device_error() reads; kernels never trap.
  *   - Results are deterministic: the same inputs give bitwise identical
  *     outputs (no floating-point atomics).
@@ -355,11 +355,13 @@ spk_status spk_mapped_host_pointer(const void* host, void** dev);
 /* Message for the last non-OK status returned on this thread ("" if none). */
 const char* spk_last_error(void);
 
-/* Synchronises the current device, then reports the first error recorded by a
+/* Synchronises the current device, then reports an error recorded by a
  * kernel since the last clear: *status = SPK_OK, SPK_ERR_TIMEOUT (a bounded
- * device wait ran out; *site says where) or SPK_ERR_ARG (kv_compact index out
- * of range).  clear != 0 resets the word.  Returns SPK_ERR_CUDA if the
- * device could not be read. */
+ * device wait ran out; *site says where) or SPK_ERR_ARG (an index out of
+ * range in kv_compact or vs_sparse_attention).  Each source file of the
+ * library keeps its own first-error word; the first set one, in a fixed
+ * order of the files, is reported.  clear != 0 resets them all.  Returns
+ * SPK_ERR_CUDA if the device could not be read. */
 spk_status spk_device_error(int* status, int* site, int clear);
 
 /* Diagnostic: y[i] = 2^t[i] as computed on the FMA pipe by the scoring
