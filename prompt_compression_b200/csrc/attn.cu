@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // per Q tile x (0: A, 1: B): s_full[x] (S ready), p_full[x] (P written, 4
   // warps), pv_done[x] (O += P V retired), o_empty[x] (O read at item end)
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
-      p_full[2], pv_done[2], o_empty[2], done_bar;
+      p_half[2], p_full[2], pv_done[2], o_empty[2], done_bar;
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
 
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
-      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kAttnSoftmaxWarps);
+      mbar_init(&s_full[s], 1); mbar_init(&p_half[s], kAttnSoftmaxWarps); mbar_init(&p_full[s], kAttnSoftmaxWarps);
       mbar_init(&pv_done[s], 1); mbar_init(&o_empty[s], kAttnSoftmaxWarps);
     }
     mbar_init(&done_bar, 1);
@@ -249,22 +249,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (x == 1) umma_commit(&k_empty[st]);
         return true;
       };
+      // O += P V in two halves: keys 64..127 as soon as the softmax has
+      // stored their P (while it works on keys 0..63), then keys 0..63
       auto issue_pv = [&](int x, uint32_t Ti, int t) -> bool {
         const int st = Ti & 1;
-        if (!mbar_wait(&p_full[x], Ti & 1, abort_v, attn_site(1, 4 + x))) return false;
+        if (!mbar_wait(&p_half[x], Ti & 1, abort_v, attn_site(1, 2 + x))) return false;
         if (x == 0 && !mbar_wait(&v_full[st], (Ti >> 1) & 1, abort_v, attn_site(1, 6))) return false;
         // the softmax group has read the previous item's O before it is restarted
         if (t == 0 && items_done > 0 && !mbar_wait(&o_empty[x], (items_done - 1) & 1, abort_v, attn_site(1, 7 + x)))
           return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(V_s + st * C::kTileBytes);
+        auto pv_steps = [&](int kk0) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // one instruction spans the head_dim / 64 column blocks (lbo apart)
-          const uint64_t v_desc = sw128_mnmajor_desc(v_base + kk * 2048, 16384);
-          umma_bf16_ts(tmem_base + x * 256 + 128, tmem_base + x * 256 + 64 + kk * 8, v_desc, idesc_pv,
-                       (t > 0 || kk > 0) ? 1u : 0u);
-        }
+          for (int kk = kk0; kk < kk0 + 4; ++kk) {
+            // one instruction spans the head_dim / 64 column blocks (lbo apart)
+            const uint64_t v_desc = sw128_mnmajor_desc(v_base + kk * 2048, 16384);
+            umma_bf16_ts(tmem_base + x * 256 + 128, tmem_base + x * 256 + 64 + kk * 8, v_desc, idesc_pv,
+                         (t > 0 || kk != 4) ? 1u : 0u);
+          }
+        };
+        pv_steps(4);
+        if (!mbar_wait(&p_full[x], Ti & 1, abort_v, attn_site(1, 4 + x))) return false;
+        tc_fence_after();
+        pv_steps(0);
         umma_commit(&pv_done[x]);
         if (x == 1) umma_commit(&v_empty[st]);
         return true;
@@ -401,6 +409,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           exp64(b0, b1, pk);
           tmem_st32(tlane + 96, pk);
         }
+        // keys 64..127 of P are in: their half of O += P V can start
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_half[x]);
         {
           uint32_t a0[32], a1[32];
           tmem_ld32(tlane, a0);
