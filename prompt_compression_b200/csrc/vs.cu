@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kVsThreads, 1)
 
   // per Q tile x (0: A, 1: B): s_full[x], p_full[x] (4 warps), pv_done[x], o_empty[x] (4 warps)
   __shared__ __align__(8) uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
-      p_full[2], pv_done[2], o_empty[2], done_bar, soft_bar;
+      p_half[2], p_full[2], pv_done[2], o_empty[2], done_bar, soft_bar;
   __shared__ uint32_t slash_tiles[kVsMaxN / 128 / 32];   // the softmax warps' item: its slash tiles
   __shared__ uint32_t prod_tiles[kVsMaxN / 128 / 32];    // the producer's item
   __shared__ uint32_t mma_tiles[kVsMaxN / 128 / 32];     // the UMMA issuer's item
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
-      mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kVsGroupWarps);
+      mbar_init(&s_full[s], 1); mbar_init(&p_half[s], kVsGroupWarps); mbar_init(&p_full[s], kVsGroupWarps);
       mbar_init(&pv_done[s], 1); mbar_init(&o_empty[s], kVsGroupWarps);
     }
     mbar_init(&done_bar, 1);
@@ -344,21 +344,29 @@ __global__ void __launch_bounds__(kVsThreads, 1)
         if (x == 1) umma_commit(&k_empty[st]);
         return true;
       };
+      // O += P V in two halves: keys 64..127 as soon as the softmax has
+      // stored their P (while it works on keys 0..63), then keys 0..63
       auto issue_pv = [&](int x, uint32_t Ti, int t) -> bool {
         const int st = Ti & 1;
-        if (!mbar_wait(&p_full[x], Ti & 1, abort_v, vs_site(1, 4 + x))) return false;
+        if (!mbar_wait(&p_half[x], Ti & 1, abort_v, vs_site(1, 2 + x))) return false;
         if (x == 0 && !mbar_wait(&v_full[st], (Ti >> 1) & 1, abort_v, vs_site(1, 6))) return false;
         if (t == 0 && items_done > 0 && !mbar_wait(&o_empty[x], (items_done - 1) & 1, abort_v, vs_site(1, 7 + x)))
           return false;
         tc_fence_after();
         const uint32_t v_base = smem_u32(V_s + st * C::kTileBytes);
+        auto pv_steps = [&](int kk0) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // one instruction spans the head_dim / 64 column blocks (lbo apart)
-          const uint64_t v_desc = vs_mnmajor_desc(v_base + kk * 2048, 16384);
-          umma_bf16_ts(tmem_base + x * 256 + 128, tmem_base + x * 256 + 64 + kk * 8, v_desc, idesc_pv,
-                       (t > 0 || kk > 0) ? 1u : 0u);
-        }
+          for (int kk = kk0; kk < kk0 + 4; ++kk) {
+            // one instruction spans the head_dim / 64 column blocks (lbo apart)
+            const uint64_t v_desc = vs_mnmajor_desc(v_base + kk * 2048, 16384);
+            umma_bf16_ts(tmem_base + x * 256 + 128, tmem_base + x * 256 + 64 + kk * 8, v_desc, idesc_pv,
+                         (t > 0 || kk != 4) ? 1u : 0u);
+          }
+        };
+        pv_steps(4);
+        if (!mbar_wait(&p_full[x], Ti & 1, abort_v, vs_site(1, 4 + x))) return false;
+        tc_fence_after();
+        pv_steps(0);
         umma_commit(&pv_done[x]);
         if (x == 1) umma_commit(&v_empty[st]);
         return true;
@@ -599,6 +607,13 @@ __global__ void __launch_bounds__(kVsThreads, 1)
           tmem_ld_wait2(a0, a1);
           exp32(a0, tlane + 64 + 32 * hh);                // masked by the first pass
           exp32(a1, tlane + 64 + 32 * hh + 16);
+          if (hh == 1) {
+            // keys 64..127 of P are in: their half of O += P V can start
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_half[x]);
+          }
         }
         l += acc2.x + acc2.y;
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
