@@ -37,7 +37,9 @@
 //               O_x's product of tile t, so O_x is quiescent once S_x(t+1)
 //               has landed.  S = Q K^T takes A and B from shared memory;
 //               O += P V takes A = P from TMEM and B = V from shared memory
-//               in its natural [key][d] layout (MN-major).
+//               in its natural [key][d] layout (MN-major), in two key halves:
+//               keys 64..127 once the softmax has stored their P (it stores
+//               those first), keys 0..63 once all of P is in.
 // TMEM (512 columns): tile A's S at 0 and O at 128, tile B's S at 256 and O
 // at 384.  No atomics: the result is deterministic.
 #include <cuda_bf16.h>

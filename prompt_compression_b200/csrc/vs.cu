@@ -33,7 +33,7 @@
 // producer warp (both heads' Q tiles, then the K/V tiles), a single-thread
 // UMMA issuer (per tile: O_A += P_A V, S_A(next), O_B += P_B V, S_B(next);
 // S = Q K^T from shared memory, O += P V with P in TMEM as bf16 and V
-// MN-major from shared memory) and eight softmax warps (thread = row; S read
+// MN-major from shared memory, keys 64..127 as soon as their P is stored) and eight softmax warps (thread = row; S read
 // in 64-column halves; lazy rescale of O when the running max moves by more
 // than 2^8).  Every role derives the same tile sequence.
 #include <cuda_bf16.h>
