@@ -485,7 +485,7 @@ def run_speckv(args, cfg, P, dev, world, rank, headline, prefill=False):
     first_flops = prefill_flops(cfg) if prefill else flops_pass
     dom = max((first_name, "score_colsum_pass"), key=lambda n: per[n])
     roofline = kernel_roofline(dom, per[dom], first_flops if dom == first_name else flops_pass, peaks,
-                               None if prefill else captured_traffic(dom, cfg.name))
+                               captured_traffic(dom, cfg.name))
     roofline["step_roofline_ms"] = max((first_flops + flops_pass) / (peak * 1e12),
                                        algorithmic_bytes(cfg) / (peaks["hbm_gbs"] * 1e9)) * 1e3
     roofline["step_frac"] = roofline["step_roofline_ms"] / ms_step
@@ -774,7 +774,8 @@ def run_vs(args, cfg, P, dev):
         "config": {"workload": cfg.name, "n": cfg.n, "n_q": cfg.n_q, "n_vertical": cfg.n_vertical,
                    "n_slash": cfg.n_slash, "l2": "inputs larger than L2; no flush"},
         "roofline": {"bound": "tensor", "kernel": "vs_attn_kernel (+ vertical gather)", "achieved": achieved,
-                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": src,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": captured_traffic("vs_attn_kernel", cfg.name), "peak_source": src,
                      "flops": "executed 128-key tiles x 2 products; useful (visible pairs) and dense-causal "
                               "figures beside it",
                      "useful_tflops": useful_flops / (ms * 1e-3) / 1e12,
@@ -784,17 +785,25 @@ def run_vs(args, cfg, P, dev):
 
 
 # ----------------------------------------------------------------- traffic bookkeeping
-# The files that define the scoring kernels (device code and their parameter block).
-SCORING_SOURCES = ("common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh")
+# The files that define each captured kernel (device code and its parameter
+# block); profiles/traffic.json records, per kernel, the sha256 of these files
+# at the capture, and the traffic is reported only while they are unchanged.
+KERNEL_SOURCES = {
+    "score_lse_pass": ("common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh"),
+    "score_colsum_pass": ("common.cuh", "exp2_poly.cuh", "score.cu", "score.cuh"),
+    "prefill_attention": ("attn.cu", "common.cuh", "exp2_poly.cuh", "score.cuh"),
+    "vs_attn_kernel": ("common.cuh", "exp2_poly.cuh", "score.cuh", "vs.cu"),
+}
+SCORING_SOURCES = KERNEL_SOURCES["score_colsum_pass"]
 
 
-def kernel_source_digest():
-    """sha256 over the scoring kernels' sources (SCORING_SOURCES); the DRAM
-    traffic captured with ncu is only reported while they are unchanged."""
+def kernel_source_digest(kernel="score_colsum_pass"):
+    """sha256 over the sources of a captured kernel (KERNEL_SOURCES); the
+    DRAM traffic captured with ncu is only reported while they are unchanged."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "prompt_compression_b200", "csrc")
-    for name in SCORING_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         h.update(name.encode())
         h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()
@@ -805,12 +814,12 @@ def captured_traffic(kernel, workload):
     profiles/traffic.json, or None when absent or captured from other sources."""
     prof = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        rec = json.load(open(prof))
+        rec = json.load(open(prof)).get("kernels", {}).get(kernel)
     except (OSError, ValueError):
         return None
-    if rec.get("source_sha256") != kernel_source_digest():
+    if not rec or kernel not in KERNEL_SOURCES or rec.get("source_sha256") != kernel_source_digest(kernel):
         return None
-    return rec.get(kernel, {}).get(workload)
+    return rec.get("workloads", {}).get(workload)
 
 
 # ----------------------------------------------------------------- e2e

@@ -17,26 +17,31 @@ def test_tensor_peak_is_the_burst_figure():
 
 
 def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
-    digest = bench.kernel_source_digest()
-    rec = {"source_sha256": digest, "score_colsum_pass": {"w": 123}}
+    digests = {k: bench.kernel_source_digest(k) for k in bench.KERNEL_SOURCES}
+    rec = {"kernels": {"score_colsum_pass": {"source_sha256": digests["score_colsum_pass"], "workloads": {"w": 123}},
+                       "vs_attn_kernel": {"source_sha256": "0" * 64, "workloads": {"w": 7}}}}
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    # the digest reads the kernel sources from ROOT too: point it back at the repository's
-    monkeypatch.setattr(bench, "kernel_source_digest", lambda: digest)
+    # the digests read the kernel sources from ROOT too: point them back at the repository's
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda k="score_colsum_pass": digests[k])
     assert bench.captured_traffic("score_colsum_pass", "w") == 123
-    assert bench.captured_traffic("score_lse_pass", "w") is None
-    rec["source_sha256"] = "0" * 64
+    assert bench.captured_traffic("score_colsum_pass", "other") is None
+    assert bench.captured_traffic("score_lse_pass", "w") is None        # not captured
+    assert bench.captured_traffic("vs_attn_kernel", "w") is None        # captured from other sources
+    rec["kernels"]["score_colsum_pass"]["source_sha256"] = "0" * 64
     (prof / "traffic.json").write_text(json.dumps(rec))
     assert bench.captured_traffic("score_colsum_pass", "w") is None
 
 
-def test_digest_covers_the_scoring_sources_only():
+def test_digests_cover_each_kernels_sources():
     a = bench.kernel_source_digest()
-    assert len(a) == 64 and a == bench.kernel_source_digest()
+    assert len(a) == 64 and a == bench.kernel_source_digest("score_colsum_pass")
     assert "decode.cu" not in bench.SCORING_SOURCES and "score.cu" in bench.SCORING_SOURCES
     assert "api.cu" not in bench.SCORING_SOURCES
+    assert "attn.cu" in bench.KERNEL_SOURCES["prefill_attention"] and "vs.cu" in bench.KERNEL_SOURCES["vs_attn_kernel"]
+    assert len({bench.kernel_source_digest(k) for k in ("score_lse_pass", "prefill_attention", "vs_attn_kernel")}) == 3
 
 
 def test_exp2_peak_from_unit_counts():
